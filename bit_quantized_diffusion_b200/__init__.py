@@ -1,0 +1,178 @@
+"""B200 (sm_100a) SVDQuant W4A4 linear and AWQ W4A16 linear.
+
+The compute lives in ``libsvdq.so`` (C ABI, include/svdq.h). This module is
+the Python binding: one function per C call, with the same name, taking torch
+CUDA tensors and marshalling pointers, sizes and the current stream. torch is
+used for device memory and streams only.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import _native as N
+from ._native import SvdqError  # noqa: F401
+
+FORMATS = {"nvfp4": N.NVFP4_G16, "int4": N.INT4_G64}
+PACK_KINDS = {"act": N.PACK_ACT, "weight": N.PACK_WEIGHT, "awq": N.PACK_AWQ}
+
+
+def _fmt(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, nbytes: int, name: str) -> None:
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {nbytes}")
+
+
+def svdq_codes_bytes(fmt, rows: int, K: int) -> int:
+    return N.load().svdq_codes_bytes(_fmt(fmt), rows, K)
+
+
+def svdq_scales_bytes(fmt, rows: int, K: int) -> int:
+    return N.load().svdq_scales_bytes(_fmt(fmt), rows, K)
+
+
+def awq_qweight_bytes(Nrows: int, K: int) -> int:
+    return N.load().awq_qweight_bytes(Nrows, K)
+
+
+def awq_sz_bytes(Nrows: int, K: int) -> int:
+    return N.load().awq_sz_bytes(Nrows, K)
+
+
+def svdq_quantize_act(X: torch.Tensor, L1t: torch.Tensor | None = None,
+                      smooth_inv: torch.Tensor | None = None, fmt="nvfp4",
+                      codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                      xl1: torch.Tensor | None = None, stream=None):
+    """Steps a1..a4 on X [M, K] bf16. Returns (codes, scales, xl1 or None)."""
+    lib = N.load()
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    r = 0 if L1t is None else L1t.shape[0]
+    f = _fmt(fmt)
+    dev = X.device
+    if codes is None:
+        codes = torch.empty(lib.svdq_codes_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(lib.svdq_scales_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    if r and xl1 is None:
+        xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
+    _need(codes, lib.svdq_codes_bytes(f, M, K), "codes")
+    _need(scales, lib.svdq_scales_bytes(f, M, K), "scales")
+    if L1t is not None and (L1t.dtype != torch.bfloat16 or tuple(L1t.shape) != (r, K)):
+        raise ValueError("L1t must be bf16 [r, K]")
+    if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
+        raise ValueError("smooth_inv must be float32 [K]")
+    if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < M * r):
+        raise ValueError("xl1 must be float32 [M, r]")
+    N.check(lib.svdq_quantize_act(f, M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(L1t),
+                                  _ptr(codes), _ptr(scales), _ptr(xl1) if r else None,
+                                  _stream(stream)), "svdq_quantize_act")
+    return codes, scales, (xl1 if r else None)
+
+
+def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int, N_: int,
+                     K: int, fmt="nvfp4", out_dtype=torch.bfloat16, Y: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Steps a5..a6: Y [M, N] = Q(X_hat) Q(R)^T + xl1 @ L2 + bias."""
+    lib = N.load()
+    r = 0 if L2 is None else L2.shape[0]
+    f = _fmt(fmt)
+    out = N.OUT_F32 if out_dtype == torch.float32 else N.OUT_BF16
+    if Y is None:
+        Y = torch.empty((M, N_), dtype=out_dtype, device=a_codes.device)
+    if Y.dtype != out_dtype or Y.dim() != 2 or Y.shape[0] != M or Y.shape[1] < N_:
+        raise ValueError("Y must be [M, >= N] of out_dtype")
+    if L2 is not None and (L2.dtype != torch.bfloat16 or tuple(L2.shape) != (r, N_)):
+        raise ValueError("L2 must be bf16 [r, N]")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N_):
+        raise ValueError("bias must be bf16 [N]")
+    _need(a_codes, lib.svdq_codes_bytes(f, M, K), "a_codes")
+    _need(a_scales, lib.svdq_scales_bytes(f, M, K), "a_scales")
+    _need(w_codes, lib.svdq_codes_bytes(f, N_, K), "w_codes")
+    _need(w_scales, lib.svdq_scales_bytes(f, N_, K), "w_scales")
+    N.check(lib.svdq_w4a4_linear(f, M, N_, K, r, _ptr(a_codes), _ptr(a_scales),
+                                 _ptr(xl1) if r else None, _ptr(w_codes), _ptr(w_scales),
+                                 _ptr(L2) if r else None, _ptr(bias), _ptr(Y), Y.shape[1], out,
+                                 _stream(stream)), "svdq_w4a4_linear")
+    return Y
+
+
+def awq_w4a16_linear(X: torch.Tensor, qweight: torch.Tensor, sz: torch.Tensor,
+                     bias: torch.Tensor | None, N_: int, group: int = 64,
+                     Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Step a7: Y [M, N] bf16 from X [M, K] bf16 and packed AWQ weights."""
+    lib = N.load()
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    if Y is None:
+        Y = torch.empty((M, N_), dtype=torch.bfloat16, device=X.device)
+    _need(qweight, lib.awq_qweight_bytes(N_, K), "qweight")
+    _need(sz, lib.awq_sz_bytes(N_, K), "sz")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N_):
+        raise ValueError("bias must be bf16 [N]")
+    N.check(lib.awq_w4a16_linear(M, N_, K, group, _ptr(X), _ptr(qweight), _ptr(sz), _ptr(bias),
+                                 _ptr(Y), _stream(stream)), "awq_w4a16_linear")
+    return Y
+
+
+def svdq_pack(kind, fmt, rows: int, K: int, plain_codes, plain_scales, plain_zeros=None,
+              tiled_codes=None, tiled_scales=None, stream=None):
+    """Plain -> tiled storage. Returns (tiled_codes, tiled_scales) as uint8 tensors."""
+    lib = N.load()
+    k = PACK_KINDS[kind] if isinstance(kind, str) else int(kind)
+    f = _fmt(fmt)
+    dev = plain_codes.device
+    if k == N.PACK_AWQ:
+        nc, ns = lib.awq_qweight_bytes(rows, K), lib.awq_sz_bytes(rows, K)
+    else:
+        nc, ns = lib.svdq_codes_bytes(f, rows, K), lib.svdq_scales_bytes(f, rows, K)
+    if tiled_codes is None:
+        tiled_codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+    if tiled_scales is None:
+        tiled_scales = torch.empty(ns, dtype=torch.uint8, device=dev)
+    _need(tiled_codes, nc, "tiled_codes")
+    _need(tiled_scales, ns, "tiled_scales")
+    N.check(lib.svdq_pack(k, f, rows, K, _ptr(plain_codes), _ptr(plain_scales), _ptr(plain_zeros),
+                          _ptr(tiled_codes), _ptr(tiled_scales), _stream(stream)), "svdq_pack")
+    return tiled_codes, tiled_scales
+
+
+def svdq_unpack(kind, fmt, rows: int, K: int, tiled_codes, tiled_scales, plain_codes,
+                plain_scales, plain_zeros=None, stream=None):
+    """Tiled -> plain storage, into caller-provided tensors."""
+    lib = N.load()
+    k = PACK_KINDS[kind] if isinstance(kind, str) else int(kind)
+    N.check(lib.svdq_unpack(k, _fmt(fmt), rows, K, _ptr(tiled_codes), _ptr(tiled_scales),
+                            _ptr(plain_codes), _ptr(plain_scales), _ptr(plain_zeros),
+                            _stream(stream)), "svdq_unpack")
+    return plain_codes, plain_scales, plain_zeros
+
+
+def svdq_check_device_status(stream=None) -> int:
+    """Synchronise the stream; return the status code (and clear the word)."""
+    return N.load().svdq_check_device_status(_stream(stream))
+
+
+def svdq_debug_wait_timeout(limit_us: int, stream=None) -> None:
+    N.check(N.load().svdq_debug_wait_timeout(limit_us, _stream(stream)), "svdq_debug_wait_timeout")

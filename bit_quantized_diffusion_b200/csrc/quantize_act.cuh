@@ -1,0 +1,353 @@
+// quantize_act.cuh -- steps a1..a4 of the SVDQuant layer in one pass over X:
+// smoothing, group scale, 4-bit quantization + packing, and the rank-r
+// down-projection x_hat @ L1 on the tensor cores (Nunchaku README, "Engine
+// design" (b): the down projection and the quantizer share their input).
+//
+// One CTA owns 128 rows and a contiguous range of 64-column chunks of X. A
+// cluster of `ksplit` CTAs covers all of K for the same 128 rows; their partial
+// x_hat @ L1 sums are added through distributed shared memory in a fixed order.
+//
+// Warp roles (18 warps):
+//   warp 0      TMA producer: X chunk [128 x 64] bf16 and L1^T chunk [r x 64] bf16,
+//               both 128-byte swizzled, into a ring of stages
+//   warp 1      tensor-memory owner and MMA issuer (one thread)
+//   warps 2..17 quantizers; warp q handles rows 8q..8q+7, lane l handles row
+//               8q + l%8 and columns 16(l/8)..16(l/8)+15 of the chunk, i.e.
+//               exactly one NVFP4 group (a quarter of an INT4 group)
+// The quantizers also write x_hat split into bf16 hi + lo (no-swizzle K-major
+// core-matrix layout) for two tcgen05 kind::f16 MMAs per K step into one f32
+// accumulator in tensor memory.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace svdq {
+
+constexpr int kQaWarps = 18;
+constexpr int kQaThreads = kQaWarps * 32;
+constexpr int kQaQuantWarps = 16;
+constexpr int kQaChunk = 64;                   // columns per stage
+constexpr int kQaXStageBytes = 128 * kQaChunk * 2;  // 16 KB
+constexpr int kQaATileBytes = 128 * kQaChunk * 2;   // one bf16 [128 x 64] tile
+
+struct QuantActParams {
+  int M, K, r;
+  int ksplit;      // CTAs per cluster along K (1, 2, 4 or 8)
+  int stages;      // ring depth
+  int m_pad;       // M rounded up to 128
+  const float* smooth_inv;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* xl1;
+  uint32_t* status;
+};
+
+struct QaSmem {
+  // byte offsets from the 1024-aligned dynamic shared memory base
+  uint32_t ring, stage_bytes, a_tiles, bars, tmem_slot;
+};
+
+__host__ __device__ inline QaSmem qa_smem_layout(int r, int stages) {
+  QaSmem s;
+  s.ring = 0;
+  s.stage_bytes = kQaXStageBytes + r * 128;
+  s.a_tiles = s.ring + stages * s.stage_bytes;
+  const uint32_t a_bytes = r > 0 ? 4 * kQaATileBytes : 0;  // 2 buffers x (hi, lo)
+  s.bars = s.a_tiles + a_bytes;
+  s.tmem_slot = s.bars + 8 * (2 * stages + 5);
+  return s;
+}
+
+__host__ inline size_t qa_smem_bytes(int r, int stages) {
+  QaSmem s = qa_smem_layout(r, stages);
+  return s.tmem_slot + 16 + 1024;  // + alignment slack
+}
+
+template <int kFmt>  // 0: NVFP4 (E2M1, UE4M3 per 16), 1: INT4 (FP16 per 64)
+__global__ void __launch_bounds__(kQaThreads, 1)
+    quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_l1, const QuantActParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const QaSmem L = qa_smem_layout(p.r, p.stages);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int NS = p.stages;
+  const int r = p.r;
+
+  const int ks = blockIdx.x % p.ksplit;
+  const int rb = blockIdx.y;
+  const int kc_total = p.K / kQaChunk;
+  const int kc0 = ks * kc_total / p.ksplit;
+  const int kc1 = (ks + 1) * kc_total / p.ksplit;
+  const int nchunks = kc1 - kc0;
+
+  auto bar_full = [&](int s) { return sbase + L.bars + 8 * s; };
+  auto bar_empty = [&](int s) { return sbase + L.bars + 8 * (NS + s); };
+  auto bar_afull = [&](int a) { return sbase + L.bars + 8 * (2 * NS + a); };
+  auto bar_aempty = [&](int a) { return sbase + L.bars + 8 * (2 * NS + 2 + a); };
+  const uint32_t bar_acc = sbase + L.bars + 8 * (2 * NS + 4);
+  auto x_stage = [&](int s) { return sbase + L.ring + s * L.stage_bytes; };
+  auto l1_stage = [&](int s) { return x_stage(s) + kQaXStageBytes; };
+  auto a_hi = [&](int a) { return sbase + L.a_tiles + a * 2 * kQaATileBytes; };
+  auto a_lo = [&](int a) { return a_hi(a) + kQaATileBytes; };
+
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
+  const uint32_t tmem_cols = r <= 32 ? 32 : (r <= 64 ? 64 : (r <= 128 ? 128 : 256));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), r > 0 ? 1 : kQaQuantWarps);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_afull(a), kQaQuantWarps);
+      mbar_init(bar_aempty(a), 1);
+    }
+    mbar_init(bar_acc, 1);
+    fence_barrier_init();
+    prefetch_tmap(&tm_x);
+    if (r > 0) prefetch_tmap(&tm_l1);
+  }
+  if (warp == 1 && r > 0) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = r > 0 ? *tmem_slot : 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (elect_one()) {
+      const uint32_t tx = kQaXStageBytes + r * 128;
+      for (int i = 0; i < nchunks; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(bar_empty(s), ((i / NS) & 1) ^ 1, p.status)) break;
+        mbar_arrive_expect_tx(bar_full(s), tx);
+        tma_load_2d(x_stage(s), &tm_x, bar_full(s), (kc0 + i) * kQaChunk, rb * 128);
+        if (r > 0) tma_load_2d(l1_stage(s), &tm_l1, bar_full(s), (kc0 + i) * kQaChunk, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (r > 0 && elect_one()) {
+      const uint32_t idesc = idesc_bf16_f32(128, r, false, false);
+      bool ok = true;
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const int s = i % NS, a = i & 1;
+        ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status) &&
+             mbar_wait(bar_afull(a), (i >> 1) & 1, p.status);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kQaChunk / 16; ++kk) {
+          // A: no-swizzle K-major, core matrices 8 rows x 16 B; K-adjacent ones
+          // 128 B apart (LBO), 8-row groups 1024 B apart (SBO); 16 K = 256 B.
+          const uint64_t ah = smem_desc(a_hi(a) + kk * 256, 128, 1024, kSwizzleNone);
+          const uint64_t al = smem_desc(a_lo(a) + kk * 256, 128, 1024, kSwizzleNone);
+          // B: L1^T rows (r of them), 128 B each, 128-byte swizzle; 16 K = 32 B.
+          const uint64_t bd = smem_desc(l1_stage(s) + kk * 32, 16, 1024, kSwizzle128B);
+          mma_f16(tmem_base, ah, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_f16(tmem_base, al, bd, idesc, 1u);
+        }
+        tc_commit(bar_empty(s));
+        tc_commit(bar_aempty(a));
+      }
+      tc_commit(bar_acc);
+    }
+  } else {
+    // ---------------------------------------------------------------- quantizers
+    const int qw = warp - 2;
+    const int row = qw * 8 + (lane & 7);
+    const int q = lane >> 3;  // which 16 columns of the chunk
+    const int m = rb * 128 + row;
+    const bool row_ok = m < p.M;
+    bool ok = true;
+    for (int i = 0; i < nchunks; ++i) {
+      const int s = i % NS;
+      const int kc = kc0 + i;
+      ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status);
+      if (!ok) break;
+      // -- load 16 bf16 of this row from the 128B-swizzled X tile
+      float xh[16];
+      {
+        const uint32_t rowbase = x_stage(s) + row * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * q + h;
+          uint32_t v0, v1, v2, v3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                       : "r"(rowbase + ((c ^ (row & 7)) << 4)));
+          const uint32_t w[4] = {v0, v1, v2, v3};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            xh[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
+            xh[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+        }
+      }
+      // -- a1: smoothing, one float32 multiply
+      if (p.smooth_inv != nullptr) {
+        const float4* sp = reinterpret_cast<const float4*>(p.smooth_inv + kc * kQaChunk + 16 * q);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 sv = __ldg(sp + j);
+          xh[4 * j + 0] = __fmul_rn(xh[4 * j + 0], sv.x);
+          xh[4 * j + 1] = __fmul_rn(xh[4 * j + 1], sv.y);
+          xh[4 * j + 2] = __fmul_rn(xh[4 * j + 2], sv.z);
+          xh[4 * j + 3] = __fmul_rn(xh[4 * j + 3], sv.w);
+        }
+      }
+      // -- a2 + a3: group scale and codes
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[j]));
+      uint32_t code_lo = 0, code_hi = 0;
+      if (kFmt == 0) {
+        const uint32_t sc = e4m3_code(__fdiv_rn(amax, 6.0f));
+        const float sval = e4m3_value(sc);
+        if (sval != 0.0f) {
+          const float rcp = __frcp_rn(sval);
+          float y0[8], y1[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            y0[j] = __fmul_rn(xh[j], rcp);
+            y1[j] = __fmul_rn(xh[8 + j], rcp);
+          }
+          code_lo = e2m1x8(y0);
+          code_hi = e2m1x8(y1);
+        }
+        // gather the row's four scale bytes into one word (lanes l, l+8, l+16, l+24)
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sc, 8);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sc, 16);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sc, 24);
+        if (q == 0) {
+          const uint32_t word = sc | (b1 << 8) | (b2 << 16) | (b3 << 24);
+          const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
+          *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
+              word;
+        }
+      } else {
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+        const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        const float sval = __half2float(hs);
+        if (sval != 0.0f) {
+          const float rcp = __frcp_rn(sval);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            int v = __float2int_rn(__fmul_rn(xh[j], rcp));
+            v = max(-7, min(7, v));
+            const uint32_t nib = static_cast<uint32_t>(v) & 0xFu;
+            if (j < 8) code_lo |= nib << (4 * j);
+            else code_hi |= nib << (4 * (j - 8));
+          }
+        }
+        if (q == 0)
+          reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] =
+              hs;
+      }
+      if (row_ok) {
+        *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + q * 8) =
+            make_uint2(code_lo, code_hi);
+      }
+      // -- a4 operand: x_hat as bf16 hi + lo for the tensor cores
+      if (r > 0) {
+        const int a = i & 1;
+        ok = mbar_wait(bar_aempty(a), ((i >> 1) & 1) ^ 1, p.status);
+        if (!ok) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float x0 = xh[8 * h + 2 * j], x1 = xh[8 * h + 2 * j + 1];
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(hb);
+            const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+            hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
+            lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
+          }
+          const uint32_t off = (row >> 3) * 1024 + (2 * q + h) * 128 + (row & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi(a) + off), "r"(hi[0]),
+                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo(a) + off), "r"(lo[0]),
+                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afull(a));
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+      }
+    }
+    // ------------------------------------------------------------ xl1 epilogue
+    if (r > 0 && ok && mbar_wait(bar_acc, 0, p.status)) {
+      tc_fence_after();
+      const int quad = warp & 3;        // tensor-memory lanes this warp may read
+      const int part = (warp - 2) >> 2;  // which quarter of the r columns
+      const int trow = quad * 32 + lane;
+      const int ncol = r / 4, c_begin = part * ncol;
+      const int rs = r + 4;  // padded row stride (floats) of the reduction buffer
+      float* red = reinterpret_cast<float*>(smem + L.ring);
+      const int tm = rb * 128 + trow;
+      for (int c = c_begin; c < c_begin + ncol; c += 4) {
+        uint32_t v[4];
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                     : "r"(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c));
+        tmem_ld_wait();
+        const float4 f = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]),
+                                     __uint_as_float(v[2]), __uint_as_float(v[3]));
+        if (p.ksplit == 1) {
+          if (tm < p.M) *reinterpret_cast<float4*>(p.xl1 + static_cast<size_t>(tm) * r + c) = f;
+        } else {
+          *reinterpret_cast<float4*>(red + trow * rs + c) = f;
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------- cluster reduction
+  if (r > 0 && p.ksplit > 1) {
+    cluster_sync();  // every CTA's partial sums are in its shared memory
+    if (warp >= 2) {
+      const int rows_per = 128 / p.ksplit;
+      const int units = rows_per * (r / 4);
+      const int rs = r + 4;
+      const uint32_t red = sbase + L.ring;
+      for (int u = threadIdx.x - 64; u < units; u += kQaQuantWarps * 32) {
+        const int trow = ks * rows_per + u / (r / 4);
+        const int c = (u % (r / 4)) * 4;
+        const uint32_t off = red + (trow * rs + c) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int pr = 0; pr < p.ksplit; ++pr) {
+          const float4 v = ld_dsmem_f4(map_peer_smem(off, pr));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int tm = rb * 128 + trow;
+        if (tm < p.M) *reinterpret_cast<float4*>(p.xl1 + static_cast<size_t>(tm) * r + c) = acc;
+      }
+    }
+    cluster_sync();  // keep shared memory alive until every peer has read it
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && r > 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace svdq

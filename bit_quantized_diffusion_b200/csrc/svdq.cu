@@ -1,0 +1,435 @@
+// svdq.cu -- the C ABI of include/svdq.h: argument checks, tensor-map
+// construction, launch configuration and the device status word.
+// All kernels live in this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/svdq.h"
+#include "awq.cuh"
+#include "pack.cuh"
+#include "quantize_act.cuh"
+#include "w4a4_gemm.cuh"
+
+namespace {
+
+using namespace svdq;
+
+__device__ uint32_t g_svdq_status;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  uint32_t* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device set-up (status word address, SM count, kernel attributes), done
+// once per device with that device current.
+svdq_status device_setup(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (g_encode == nullptr) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return SVDQ_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    void* st = nullptr;
+    if (cudaGetSymbolAddress(&st, g_svdq_status) != cudaSuccess) return SVDQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    const int max_smem = 232448;
+    if (cudaFuncSetAttribute(quantize_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(quantize_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kGmSmemBytes)) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    d.status = static_cast<uint32_t*>(st);
+    d.ready = true;
+  }
+  *out = &d;
+  return SVDQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svdq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool rank_ok(int r) { return r == 0 || (r % 16 == 0 && r >= 16 && r <= 256); }
+
+size_t pad128(int rows) { return (static_cast<size_t>(rows) + 127) / 128 * 128; }
+
+unsigned grid_for(size_t n, unsigned threads) {
+  size_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 65535u * 8u) b = 65535u * 8u;
+  return static_cast<unsigned>(b);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svdq_status_str(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported by this build";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+  }
+  return "unknown status";
+}
+
+int svdq_version(void) { return 100; }
+
+size_t svdq_codes_bytes(svdq_format f, int rows, int K) {
+  if ((f != SVDQ_NVFP4_G16 && f != SVDQ_INT4_G64) || rows < 1 || K < 64 || K % 64) return 0;
+  return static_cast<size_t>(rows) * (K / 2);
+}
+
+size_t svdq_scales_bytes(svdq_format f, int rows, int K) {
+  if (rows < 1 || K < 64 || K % 64) return 0;
+  if (f == SVDQ_NVFP4_G16) return pad128(rows) * (K / 16);
+  if (f == SVDQ_INT4_G64) return pad128(rows) * (K / 64) * 2;
+  return 0;
+}
+
+size_t awq_qweight_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 2);
+}
+
+size_t awq_sz_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 64) * 4;
+}
+
+svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
+                              const float* smooth_inv, const void* L1t, void* codes,
+                              void* scales, float* xl1, svdq_stream_t stream) {
+  if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 64 || K % 64 || !rank_ok(r) || ldx < K) return SVDQ_ERR_INVALID_ARG;
+  if (X == nullptr || codes == nullptr || scales == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (xl1 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || ldx % 8 ||
+      (smooth_inv && !aligned16(smooth_inv)) || (L1t && !aligned16(L1t)) ||
+      (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+
+  CUtensorMap tm_x, tm_l1;
+  if (!make_tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(ldx) * 2,
+                    64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  if (r > 0) {
+    if (!make_tmap_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, K, r,
+                      static_cast<uint64_t>(K) * 2, 64, r, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l1 = tm_x;  // unused
+  }
+
+  const int row_blocks = (M + 127) / 128;
+  const int kc_total = K / 64;
+  int ksplit = 1;
+  while (ksplit * 2 <= 8 && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= d->num_sms)
+    ksplit *= 2;
+  const int stage_bytes = kQaXStageBytes + r * 128;
+  const int avail = 232448 - 1024 - 256 - (r > 0 ? 4 * kQaATileBytes : 0);
+  int stages = avail / stage_bytes;
+  if (stages > 8) stages = 8;
+  if (stages < 2) return SVDQ_ERR_UNSUPPORTED;
+  // the ring is reused for the cross-CTA reduction of the [128 x r] partial sums
+  if (r > 0 && 128 * (r + 4) * 4 > stages * stage_bytes) return SVDQ_ERR_UNSUPPORTED;
+
+  QuantActParams p;
+  p.M = M;
+  p.K = K;
+  p.r = r;
+  p.ksplit = ksplit;
+  p.stages = stages;
+  p.m_pad = static_cast<int>(pad128(M));
+  p.smooth_inv = smooth_inv;
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.xl1 = xl1;
+  p.status = d->status;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ksplit, row_blocks, 1);
+  cfg.blockDim = dim3(kQaThreads, 1, 1);
+  cfg.dynamicSmemBytes = qa_smem_bytes(r, stages);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (r > 0 && ksplit > 1) ? 1 : 0;
+  cudaError_t e = format == SVDQ_NVFP4_G16
+                      ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<0>, tm_x, tm_l1, p)
+                      : cudaLaunchKernelEx(&cfg, quantize_act_kernel<1>, tm_x, tm_l1, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
+                             const void* a_scales, const float* xl1, const void* w_codes,
+                             const void* w_scales, const void* L2, const void* bias, void* Y,
+                             int ldy, svdq_out out, svdq_stream_t stream) {
+  if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+  if (out != SVDQ_OUT_BF16 && out != SVDQ_OUT_F32) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 16 || N % 16 || K < 64 || K % 64 || !rank_ok(r) || ldy < N)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !Y) return SVDQ_ERR_INVALID_ARG;
+  if ((r > 0) != (xl1 != nullptr) || (r > 0) != (L2 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  const int esz = out == SVDQ_OUT_F32 ? 4 : 2;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(Y) || (xl1 && !aligned16(xl1)) || (L2 && !aligned16(L2)) ||
+      (bias && !aligned16(bias)) || (static_cast<size_t>(ldy) * esz) % 16)
+    return SVDQ_ERR_ALIGNMENT;
+  if (format != SVDQ_NVFP4_G16) return SVDQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+
+  CUtensorMap tm_a, tm_b, tm_l2;
+  if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, kGmBKBytes,
+                    kGmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, kGmBKBytes,
+                    kGmBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  if (r > 0) {
+    if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, N, r,
+                      static_cast<uint64_t>(N) * 2, 64, kGmLrK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l2 = tm_a;
+  }
+  GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.a_scales = static_cast<const uint8_t*>(a_scales);
+  p.w_scales = static_cast<const uint8_t*>(w_scales);
+  p.xl1 = xl1;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = Y;
+  p.ldy = ldy;
+  p.out_f32 = out == SVDQ_OUT_F32;
+  p.status = d->status;
+  dim3 grid((M + kGmBM - 1) / kGmBM, (N + kGmBN - 1) / kGmBN, 1);
+  w4a4_nvfp4_gemm_kernel<<<grid, kGmThreads, kGmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      tm_a, tm_b, tm_l2, p);
+  return launch_status();
+}
+
+svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, const void* qweight,
+                             const void* sz, const void* bias, void* Y, svdq_stream_t stream) {
+  if (group != 64 || M < 1 || M > kAwqMaxM || N < 1 || K < 64 || K % 64)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!X || !qweight || !sz || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(qweight) || !aligned16(sz) || !aligned16(Y) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 1)))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  AwqParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.qweight = static_cast<const uint4*>(qweight);
+  p.sz = static_cast<const uint32_t*>(sz);
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  const int nblocks = (N + 15) / 16;
+  dim3 grid((nblocks + 3) / 4);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch ((M + 7) / 8) {
+    case 1: awq_gemv_kernel<1><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 2: awq_gemv_kernel<2><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 3: awq_gemv_kernel<3><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 4: awq_gemv_kernel<4><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 5: awq_gemv_kernel<5><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 6: awq_gemv_kernel<6><<<grid, kAwqThreads, 0, s>>>(p); break;
+    case 7: awq_gemv_kernel<7><<<grid, kAwqThreads, 0, s>>>(p); break;
+    default: awq_gemv_kernel<8><<<grid, kAwqThreads, 0, s>>>(p); break;
+  }
+  return launch_status();
+}
+
+svdq_status svdq_pack(svdq_pack_kind kind, svdq_format format, int rows, int K,
+                      const void* plain_codes, const void* plain_scales, const void* plain_zeros,
+                      void* tiled_codes, void* tiled_scales, svdq_stream_t stream) {
+  if (rows < 1 || K < 64 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!plain_codes || !plain_scales || !tiled_codes || !tiled_scales) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(plain_codes) || !aligned16(tiled_codes) || !aligned16(tiled_scales) ||
+      (reinterpret_cast<uintptr_t>(plain_scales) & 1))
+    return SVDQ_ERR_ALIGNMENT;
+  if (kind != SVDQ_PACK_ACT && kind != SVDQ_PACK_WEIGHT && kind != SVDQ_PACK_AWQ)
+    return SVDQ_ERR_INVALID_ARG;
+  if (kind == SVDQ_PACK_AWQ) {
+    if (plain_zeros == nullptr || (reinterpret_cast<uintptr_t>(plain_zeros) & 1)) return SVDQ_ERR_INVALID_ARG;
+  } else if (plain_zeros != nullptr || (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64)) {
+    return SVDQ_ERR_INVALID_ARG;
+  }
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned T = 256;
+  if (kind == SVDQ_PACK_ACT || kind == SVDQ_PACK_WEIGHT) {
+    if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
+    if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+    const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
+    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(plain_codes),
+                                                     static_cast<uint4*>(tiled_codes), n16);
+    if (format == SVDQ_NVFP4_G16) {
+      const size_t n = pad128(rows) * (K / 16);
+      pack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
+          static_cast<const uint8_t*>(plain_scales), static_cast<uint8_t*>(tiled_scales), rows, K);
+    } else {
+      const size_t n = pad128(rows) * (K / 64);
+      pack_int4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
+          static_cast<const uint16_t*>(plain_scales), static_cast<uint16_t*>(tiled_scales), rows,
+          K);
+    }
+    return launch_status();
+  }
+  if (kind == SVDQ_PACK_AWQ) {
+    if (plain_zeros == nullptr || (reinterpret_cast<uintptr_t>(plain_zeros) & 1))
+      return SVDQ_ERR_INVALID_ARG;
+    const size_t nw = (static_cast<size_t>(rows) + 15) / 16 * (K / 64) * 128;
+    pack_awq_qweight_kernel<<<grid_for(nw, T), T, 0, s>>>(
+        static_cast<const uint8_t*>(plain_codes), static_cast<uint32_t*>(tiled_codes), rows, K);
+    const size_t ns = (static_cast<size_t>(rows) + 15) / 16 * (K / 64) * 16;
+    pack_awq_sz_kernel<<<grid_for(ns, T), T, 0, s>>>(
+        static_cast<const uint16_t*>(plain_scales), static_cast<const uint16_t*>(plain_zeros),
+        static_cast<uint32_t*>(tiled_scales), rows, K);
+    return launch_status();
+  }
+  return SVDQ_ERR_INVALID_ARG;
+}
+
+svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K,
+                        const void* tiled_codes, const void* tiled_scales, void* plain_codes,
+                        void* plain_scales, void* plain_zeros, svdq_stream_t stream) {
+  if (rows < 1 || K < 64 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!plain_codes || !plain_scales || !tiled_codes || !tiled_scales) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(plain_codes) || !aligned16(tiled_codes) || !aligned16(tiled_scales) ||
+      (reinterpret_cast<uintptr_t>(plain_scales) & 1))
+    return SVDQ_ERR_ALIGNMENT;
+  if (kind != SVDQ_PACK_ACT && kind != SVDQ_PACK_WEIGHT && kind != SVDQ_PACK_AWQ)
+    return SVDQ_ERR_INVALID_ARG;
+  if (kind == SVDQ_PACK_AWQ) {
+    if (plain_zeros == nullptr || (reinterpret_cast<uintptr_t>(plain_zeros) & 1)) return SVDQ_ERR_INVALID_ARG;
+  } else if (plain_zeros != nullptr || (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64)) {
+    return SVDQ_ERR_INVALID_ARG;
+  }
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned T = 256;
+  if (kind == SVDQ_PACK_ACT || kind == SVDQ_PACK_WEIGHT) {
+    if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
+    if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+    const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
+    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(tiled_codes),
+                                                     static_cast<uint4*>(plain_codes), n16);
+    if (format == SVDQ_NVFP4_G16) {
+      const size_t n = static_cast<size_t>(rows) * (K / 16);
+      unpack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
+          static_cast<const uint8_t*>(tiled_scales), static_cast<uint8_t*>(plain_scales), rows, K);
+    } else {
+      const size_t n = static_cast<size_t>(rows) * (K / 64);
+      unpack_int4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
+          static_cast<const uint16_t*>(tiled_scales), static_cast<uint16_t*>(plain_scales), rows,
+          K);
+    }
+    return launch_status();
+  }
+  if (kind == SVDQ_PACK_AWQ) {
+    if (plain_zeros == nullptr || (reinterpret_cast<uintptr_t>(plain_zeros) & 1))
+      return SVDQ_ERR_INVALID_ARG;
+    const size_t nb = static_cast<size_t>(rows) * (K / 2);
+    unpack_awq_qweight_kernel<<<grid_for(nb, T), T, 0, s>>>(
+        static_cast<const uint32_t*>(tiled_codes), static_cast<uint8_t*>(plain_codes), rows, K);
+    const size_t ns = static_cast<size_t>(rows) * (K / 64);
+    unpack_awq_sz_kernel<<<grid_for(ns, T), T, 0, s>>>(
+        static_cast<const uint32_t*>(tiled_scales), static_cast<uint16_t*>(plain_scales),
+        static_cast<uint16_t*>(plain_zeros), rows, K);
+    return launch_status();
+  }
+  return SVDQ_ERR_INVALID_ARG;
+}
+
+svdq_status svdq_check_device_status(svdq_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_svdq_status, sizeof(v)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_svdq_status, &zero, sizeof(zero)) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+  }
+  return (v & kStatusTimeout) ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+svdq_status svdq_debug_wait_timeout(int limit_us, svdq_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SVDQ_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  debug_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      d->status, static_cast<uint64_t>(limit_us) * 1000ull);
+  return launch_status();
+}
+
+}  // extern "C"

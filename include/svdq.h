@@ -1,0 +1,199 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 / AWQ W4A16 linear library.
+ *
+ * The layer (Nunchaku README, "Method": SVDQuant's three stages; "Engine design":
+ * the 16-bit low-rank branch beside the 4-bit GEMM):
+ *
+ *     Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + bias,   X_hat = X diag(smooth_inv)
+ *
+ * Q is NVFP4 (E2M1 codes, one unsigned E4M3 scale per 16 values along K) or
+ * INT4 (symmetric, one FP16 scale per 64 values along K) -- the Diffusers blog,
+ * "quantization_config": svdq_w4a4 {precision, group_size, rank} and awq_w4a16
+ * {precision int4, group_size 64}.
+ *
+ * Conventions for every call:
+ *  - Memory: the caller allocates and owns every buffer. Pointers named as device
+ *    pointers must be device memory, 16-byte aligned. The library allocates
+ *    nothing, frees nothing and synchronises nothing (svdq_check_device_status
+ *    is the one call that synchronises its stream).
+ *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream). All
+ *    work is enqueued on it; calls return before the GPU work finishes.
+ *  - Errors: argument errors are detected on the host before any launch and
+ *    returned synchronously; nothing is launched then. A failed launch returns
+ *    SVDQ_ERR_CUDA. A kernel whose bounded wait ran out records it in a device
+ *    status word, read (and cleared) by svdq_check_device_status.
+ *  - Matrices are row-major. bf16/fp16 are IEEE-style 16-bit patterns.
+ *  - Shapes: M >= 1; K % 64 == 0; N % 16 == 0; r == 0 or (r % 16 == 0 and r <= 256).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* svdq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1, /* a shape, pointer or enum is out of contract */
+  SVDQ_ERR_ALIGNMENT = 2,   /* a pointer or leading dimension is not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED = 3, /* valid request this build does not implement */
+  SVDQ_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  SVDQ_ERR_TIMEOUT = 5      /* a kernel's bounded wait ran out (device status word) */
+} svdq_status;
+
+typedef enum {
+  SVDQ_NVFP4_G16 = 0, /* E2M1 codes, UE4M3 scale per 16 along K */
+  SVDQ_INT4_G64 = 1   /* int4 codes in [-7, 7], FP16 scale per 64 along K */
+} svdq_format;
+
+typedef enum { SVDQ_OUT_BF16 = 0, SVDQ_OUT_F32 = 1 } svdq_out;
+
+typedef enum {
+  SVDQ_PACK_ACT = 0,    /* activation codes + scales */
+  SVDQ_PACK_WEIGHT = 1, /* residual-weight codes + scales (same layouts as ACT) */
+  SVDQ_PACK_AWQ = 2     /* AWQ qweight + scales + zeros */
+} svdq_pack_kind;
+
+/* Human-readable name of a status code (static storage). */
+const char* svdq_status_str(svdq_status status);
+
+/* Library ABI version (major * 100 + minor). */
+int svdq_version(void);
+
+/*
+ * Buffer sizes in bytes of the storage formats below. Codes are plain row-major
+ * packed nibbles, K contiguous, element 2j in the low nibble, 2j+1 in the high
+ * nibble (INT4 as two's complement): rows * K / 2 bytes.
+ * Scales ("tiled"):
+ *  - NVFP4: rows padded to 128; for row m and scale column j = k/16 the byte sits
+ *    in 512-byte atom a = (m/128) * (K/64) + j/4 at offset
+ *    (m%32)*16 + ((m%128)/32)*4 + j%4. This is the order tcgen05.cp copies into
+ *    tensor memory for the block-scaled MMA, so the kernels read it unchanged.
+ *  - INT4: FP16 at [K/64][rows padded to 128] (group-major), padding 0.
+ * Returns 0 for an invalid request.
+ */
+size_t svdq_codes_bytes(svdq_format format, int rows, int K);
+size_t svdq_scales_bytes(svdq_format format, int rows, int K);
+
+/* AWQ storage (see svdq_pack): fragment-ordered qweight and interleaved (scale, zero). */
+size_t awq_qweight_bytes(int N, int K);
+size_t awq_sz_bytes(int N, int K);
+
+/*
+ * svdq_quantize_act -- steps a1..a4: smooth, group-scale, quantize + pack the
+ * activations, and the rank-r down-projection of the smoothed activations, in
+ * one pass over X (Nunchaku README, "Engine design" (b): the down projection and
+ * the quantizer read the same input).
+ *
+ *   x_hat[m,k] = RN32(X[m,k] * smooth_inv[k])             (smooth_inv NULL -> x_hat = X)
+ *   NVFP4: s = UE4M3(RN32(amax16 / 6)), q = E2M1(RN32(x_hat * RN32(1 / s)))
+ *   INT4:  s = FP16(RN32(amax64 / 7)),  q = clamp(rint(RN32(x_hat * RN32(1 / s))), -7, 7)
+ *   a group whose decoded scale is 0 stores scale 0 and codes 0
+ *   xl1[m,:] = x_hat[m,:] @ L1                            (float32 output)
+ *
+ * X          device, bf16 [M, ldx] (first K columns used), ldx % 8 == 0
+ * smooth_inv device, float32 [K], or NULL
+ * L1t        device, bf16 [r, K]: L1 stored transposed (K contiguous); NULL iff r == 0
+ * codes      device, svdq_codes_bytes(format, M, K) bytes, written
+ * scales     device, svdq_scales_bytes(format, M, K) bytes, written (padding rows too)
+ * xl1        device, float32 [M, r], written; NULL iff r == 0
+ * Codes and scales are bit-exact functions of the inputs. xl1 is computed on the
+ * tensor cores with x_hat split into two bf16 terms (hi + lo) and float32
+ * accumulation. This call also serves as the weight quantizer (residual R given
+ * as bf16, smooth_inv NULL, r 0).
+ */
+svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
+                              const float* smooth_inv, const void* L1t, void* codes,
+                              void* scales, float* xl1, svdq_stream_t stream);
+
+/*
+ * svdq_w4a4_linear -- steps a5..a6: the 4-bit GEMM with the low-rank
+ * up-projection and bias accumulated into the same tensor-memory accumulator
+ * (Nunchaku README, "Engine design" (b): the up projection and the 4-bit
+ * compute share the output).
+ *
+ *   Y[m,n] = sum_g s_a[m,g] s_w[n,g] sum_{k in g} q_a[m,k] q_w[n,k]
+ *          + sum_j xl1[m,j] L2[j,n] + bias[n]
+ *
+ * a_codes, a_scales  device, activation codes/scales from svdq_quantize_act (M rows)
+ * xl1                device, float32 [M, r]; NULL iff r == 0
+ * w_codes, w_scales  device, weight codes/scales in the same formats (N rows)
+ * L2                 device, bf16 [r, N]; NULL iff r == 0
+ * bias               device, bf16 [N], or NULL
+ * Y                  device, [M, ldy] bf16 (out = SVDQ_OUT_BF16) or float32, ldy >= N,
+ *                    ldy * element size % 16 == 0
+ * The low-rank product uses xl1 split into two bf16 terms; accumulation is float32.
+ */
+svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
+                             const void* a_scales, const float* xl1, const void* w_codes,
+                             const void* w_scales, const void* L2, const void* bias, void* Y,
+                             int ldy, svdq_out out, svdq_stream_t stream);
+
+/*
+ * awq_w4a16_linear -- step a7, the AWQ W4A16 linear for small-M modulation
+ * projections (Diffusers blog, "From SVDQuant to Nunchaku Lite": awq_w4a16 for
+ * the memory-bound adaptive-norm projections).
+ *
+ *   Y[m,n] = sum_k X[m,k] (q[n,k] - z[n,k/64]) s[n,k/64] + bias[n]
+ *
+ * X        device, bf16 [M, K] (row-major, K contiguous), 1 <= M <= 64
+ * qweight  device, awq_qweight_bytes(N, K) bytes, fragment order from svdq_pack(AWQ)
+ * sz       device, awq_sz_bytes(N, K) bytes, interleaved (s, z) from svdq_pack(AWQ)
+ * bias     device, bf16 [N] or NULL
+ * Y        device, bf16 [M, N]
+ * group must be 64. Accumulation is float32; (q - z) is exact in bf16 and each
+ * group's sum is scaled by s in float32.
+ */
+svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, const void* qweight,
+                             const void* sz, const void* bias, void* Y, svdq_stream_t stream);
+
+/*
+ * svdq_pack / svdq_unpack -- convert between plain and tiled storage
+ * (unpack(pack(x)) == x bit for bit).
+ *
+ * ACT / WEIGHT: plain_codes [rows, K/2] bytes -> tiled codes (the same bytes);
+ *   plain_scales: NVFP4 uint8 [rows, K/16] E4M3 codes, INT4 fp16 [rows, K/64]
+ *   -> tiled scales (layouts above). plain_zeros must be NULL.
+ * AWQ: plain_codes = qweight [N, K/2] (element 2j low nibble, values 0..15),
+ *   plain_scales = bf16 [N, K/64], plain_zeros = bf16 [N, K/64]
+ *   -> tiled_codes (awq_qweight_bytes), tiled_scales (awq_sz_bytes). format ignored.
+ *   Fragment order: for 16-row block b and group g, 32 lanes x 16 bytes; lane t
+ *   (r0 = t/4, c0 = 2(t%4)) holds words w_j, j = 0..3 (k = 64g + 16j + ...); nibble
+ *   slot s of w_j holds W[r0 + {0,8,0,8,0,8,0,8}[s]][c0 + {0,0,8,8,1,1,9,9}[s]].
+ *   (s, z) pairs sit at [N/16][K/64][16][2].
+ * All pointers device; rows of padding are written as zeros.
+ */
+svdq_status svdq_pack(svdq_pack_kind kind, svdq_format format, int rows, int K,
+                      const void* plain_codes, const void* plain_scales, const void* plain_zeros,
+                      void* tiled_codes, void* tiled_scales, svdq_stream_t stream);
+svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K,
+                        const void* tiled_codes, const void* tiled_scales, void* plain_codes,
+                        void* plain_scales, void* plain_zeros, svdq_stream_t stream);
+
+/*
+ * svdq_check_device_status -- synchronises `stream`, then reads and clears the
+ * device status word of the current device. Returns SVDQ_ERR_TIMEOUT if any
+ * kernel's bounded wait ran out since the last check, SVDQ_ERR_CUDA if the
+ * stream reported an error, else SVDQ_OK.
+ */
+svdq_status svdq_check_device_status(svdq_stream_t stream);
+
+/*
+ * svdq_debug_wait_timeout -- diagnostics: launches one CTA that waits on a
+ * barrier no one arrives at, with a bound of `limit_us` microseconds, no copy in
+ * flight. The wait runs out, the kernel records SVDQ_ERR_TIMEOUT in the status
+ * word and returns normally. Used to test the failure-detection path without
+ * faulting or hanging the GPU. 1 <= limit_us <= 1000000.
+ */
+svdq_status svdq_debug_wait_timeout(int limit_us, svdq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */
