@@ -1,0 +1,488 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 hot path on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  1. svdq_quantize_act  -- smoothing, NVFP4 quantization and the rank-32
+                           down-projection of X [4608, 3072] (FLUX-like QKV input)
+  2. svdq_w4a4_linear   -- the NVFP4 GEMM to N = 9216 with the fused low-rank
+                           up-projection and bias
+  3. awq_w4a16_linear   -- the AWQ W4A16 adaLN modulation projection
+                           (M = 4, K = 3072, N = 18432)
+The metric is TFLOP/s over the step: 2MNK + 2Mr(K+N) for the SVDQ layer plus
+2MNK for the AWQ layer, divided by the device time of the step. L2 is flushed
+(a 256 MiB write) before every step, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same layer on
+its own token batch (data parallel, no collective on the data path); the
+reported value is the work of all ranks over the slowest rank's device time.
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "SVDQ W4A4 linear TFLOPS (NVFP4, r=32) and % of FP4 tensor roofline"
+UNIT = "TFLOP/s"
+SHAPE = WL.QKV
+AWQ = WL.AWQ_MOD
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+
+
+def layer_flops(M: int, K: int, N: int, r: int) -> float:
+    return 2.0 * M * N * K + 2.0 * M * r * (K + N)
+
+
+def step_flops() -> float:
+    return layer_flops(SHAPE.M, SHAPE.K, SHAPE.N, SHAPE.r) + 2.0 * AWQ.M * AWQ.N * AWQ.K
+
+
+def quantize_bytes(M: int, K: int, r: int) -> float:
+    """Algorithmic HBM bytes of svdq_quantize_act (NVFP4)."""
+    return 2.0 * M * K + M * K / 2 + M * K / 16 + 4.0 * M * r + 2.0 * K * r + 4.0 * K
+
+
+def awq_bytes(M: int, K: int, N: int) -> float:
+    return N * K / 2 + N * (K / 64) * 4 + 2.0 * M * K + 2.0 * M * N + 2.0 * N
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantized_diffusion_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch of `kernel` recorded from an ncu capture in
+    profiles/, if the capture was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    for line in open(path):
+        parts = line.strip().strip("|").split("|")
+        if len(parts) >= 3 and parts[0].strip() == kernel and parts[2].strip() == sha:
+            return float(parts[1])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            pr = torch.cuda.get_device_properties(cuda_index)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:  # NVML missing: report no clocks rather than guess
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = self._reasons(self._h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, rs in self.samples:
+            bits |= rs
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_sample_step(rows: int, cols: int, awq_rows: int, host: dict) -> float:
+    """The CPU oracle, as it stands, on a sample of the same step: `rows` token
+    rows x `cols` output features of the SVDQ layer (a1..a6) and `awq_rows`
+    output features of the AWQ layer (a7). Returns the sample's flops."""
+    from oracle import awq as OA
+    from oracle import svdq as S
+    bias = None if host["bias_bits"] is None else host["bias_bits"][:cols]
+    fwd = S.svdq_forward("nvfp4", host["x_bits"][:rows], host["smooth_inv"], host["L1"],
+                         host["L2"][:, :cols], host["w_codes"][:cols], host["w_scales"][:cols], bias)
+    assert fwd["Y"].shape == (rows, cols)
+    ya = OA.linear(host["xa"], host["q"][:awq_rows], host["s"][:awq_rows], host["z"][:awq_rows])
+    assert ya.shape == (AWQ.M, awq_rows)
+    return (2.0 * rows * cols * SHAPE.K + 2.0 * rows * SHAPE.r * (SHAPE.K + cols)
+            + 2.0 * AWQ.M * awq_rows * AWQ.K)
+
+
+def sample_text(rows: int, cols: int, awq_rows: int) -> str:
+    return (f"{rows} of {SHAPE.M} token rows x {cols} of {SHAPE.N} output features of the QKV "
+            f"layer (a1..a6, weights dequantized per call) + {awq_rows} of {AWQ.N} AWQ output "
+            f"features (a7)")
+
+
+def oracle_inputs_from_device(dev: dict) -> dict:
+    """Host copies of the prepared layer, in the oracle's plain formats."""
+    from oracle import formats as F
+    from oracle import layout as LO
+    from oracle import svdq as S
+    w = dev["svdq"]
+    K, N, r = SHAPE.K, SHAPE.N, SHAPE.r
+    bits = lambda t: t.view(__import__("torch").int16).cpu().numpy().view(np.uint16)  # noqa: E731
+    wq = S.unpack_nibbles(w["w_codes"].cpu().numpy().reshape(N, K // 2))
+    ws = LO.untile_nvfp4_scales(w["w_scales"].cpu().numpy(), N, K)
+    a = dev["awq_plain"]
+    return {"x_bits": dev["x_bits"], "smooth_inv": w["smooth_inv"].cpu().numpy().astype(np.float64),
+            "L1": F.bf16_from_bits(bits(w["L1"])), "L2": F.bf16_from_bits(bits(w["L2"])),
+            "w_codes": wq, "w_scales": ws, "bias_bits": dev["bias_bits"],
+            "xa": F.bf16_from_bits(dev["xa_bits"]), "q": a["q"], "s": a["s"], "z": a["z"]}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(host: dict, budget_s: float, rows: int, cols: int,
+                awq_rows: int) -> tuple[float, float, int]:
+    """Repeat the oracle sample until `budget_s` elapses; returns (flops, seconds, reps)."""
+    flops, t0, reps = 0.0, time.perf_counter(), 0
+    while True:
+        flops += oracle_sample_step(rows, cols, awq_rows, host)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return flops, time.perf_counter() - t0, reps
+
+
+def awq_plain_host(w_bits: np.ndarray) -> dict:
+    from oracle import awq as OA
+    from oracle import formats as F
+    q, s, z = OA.quantize_weight(F.bf16_from_bits(w_bits))
+    return {"q": q, "s": s, "z": z}
+
+
+def run_reference(args, rank: int) -> None:
+    """--impl reference: the oracle on the host cores, bounded samples of the same step."""
+    if rank != 0:
+        return
+    import torch  # noqa: F401  (only for symmetry of the environment)
+    from oracle import formats as F
+    from oracle import prep as P
+    from oracle import svdq as S
+    d = WL.svdq_inputs(SHAPE)
+    pr = P.prepare_svdq_layer("nvfp4", d["X"], d["W"], SHAPE.r)
+    da = WL.awq_inputs(AWQ)
+    ap = awq_plain_host(da["W"])
+    host = {"x_bits": d["X"], "smooth_inv": pr["smooth_inv"], "L1": pr["L1"], "L2": pr["L2"],
+            "w_codes": pr["w_codes"], "w_scales": pr["w_scales"], "bias_bits": d["bias"],
+            "xa": F.bf16_from_bits(da["X"]), **ap}
+    # size each step so that warmup + steps fit in about two minutes
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    rows, cols, awq_rows = 8, 1152, 1152
+    t0 = time.perf_counter()
+    oracle_sample_step(rows, cols, awq_rows, host)
+    base = time.perf_counter() - t0
+    if base > per_step:
+        shrink = max(1, int(np.ceil(base / per_step)))
+        cols, awq_rows = max(16, cols // shrink), max(16, awq_rows // shrink)
+    for _ in range(args.warmup):
+        oracle_sample_step(rows, cols, awq_rows, host)
+    flops, t0 = 0.0, time.perf_counter()
+    for _ in range(args.steps):
+        flops += oracle_sample_step(rows, cols, awq_rows, host)
+    secs = time.perf_counter() - t0
+    value = flops / secs / 1e12
+    cores = blas_threads()
+    sample = sample_text(rows, cols, awq_rows) + " per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_block(args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def config_block(n_gpus: int) -> dict:
+    return {"workload": f"{SHAPE.name}: SVDQ W4A4 linear M={SHAPE.M} K={SHAPE.K} N={SHAPE.N} "
+                        f"r={SHAPE.r} NVFP4 g16 + bias; AWQ W4A16 M={AWQ.M} K={AWQ.K} N={AWQ.N} g64",
+            "M": SHAPE.M, "K": SHAPE.K, "N": SHAPE.N, "r": SHAPE.r, "format": "nvfp4_g16",
+            "awq": {"M": AWQ.M, "K": AWQ.K, "N": AWQ.N, "group": AWQ.group},
+            "l2": "flushed before every step (256 MiB write, outside the timed events)",
+            "parallelism": f"dp{n_gpus} (independent token batches per GPU, no collective)"}
+
+
+# ------------------------------------------------------------------- our arm
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle time for the cpu_baseline leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_diffusion_b200 as bq
+    from bit_quantized_diffusion_b200 import prep
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+
+    # ---------------------------------------------------------------- inputs
+    d = WL.svdq_inputs(SHAPE)
+    x_bits = d["X"] if rank == 0 else np.roll(d["X"], 37 * rank, axis=0)
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    X = to_dev(x_bits)
+    W = to_dev(d["W"])
+    bias = to_dev(d["bias"])
+    x_absmax = X.float().abs().amax(dim=0)
+    svdq_w = prep.prepare_svdq_weights(W, x_absmax, SHAPE.r, "nvfp4")
+    da = WL.awq_inputs(AWQ)
+    Xa = to_dev(da["X"])
+    awq_w = prep.prepare_awq_weights(to_dev(da["W"]))
+    bias_a = to_dev(da["bias"])
+    del W
+    M, K, N, r = SHAPE.M, SHAPE.K, SHAPE.N, SHAPE.r
+    codes = torch.empty(bq.svdq_codes_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
+    scales = torch.empty(bq.svdq_scales_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
+    xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    Ya = torch.empty((AWQ.M, AWQ.N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        bq.svdq_quantize_act(X, svdq_w["L1s"], svdq_w["smooth_inv"], codes=codes, scales=scales,
+                             xl1=xl1, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        bq.svdq_w4a4_linear(codes, scales, xl1, svdq_w["w_codes"], svdq_w["w_scales"], svdq_w["L2"],
+                            bias, M, N, K, Y=Y, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        bq.awq_w4a16_linear(Xa, awq_w["qweight"], awq_w["sz"], bias_a, AWQ.N, Y=Ya, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if bq.svdq_check_device_status() != 0:
+        raise SystemExit("device status reported a timeout during warm-up")
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev_s = [mk() for _ in range(args.steps)]
+    ev_e = [mk() for _ in range(args.steps)]
+    ev_k = [(mk(), mk()) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            ev_s[i].record(stream)
+            step(ev_k[i])
+            ev_e[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s, ev_e))
+    k1_ms = sum(a.elapsed_time(b[0]) for a, b in zip(ev_s, ev_k)) / args.steps
+    k2_ms = sum(b[0].elapsed_time(b[1]) for b in ev_k) / args.steps
+    k3_ms = sum(b[1].elapsed_time(e) for b, e in zip(ev_k, ev_e)) / args.steps
+    status = bq.svdq_check_device_status()
+
+    # ----------------------------------------------- end to end, host buffers
+    Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+    Xh.copy_(X)
+    Xah = torch.empty(Xa.shape, dtype=Xa.dtype, pin_memory=True)
+    Xah.copy_(Xa)
+    Yh = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+    Yah = torch.empty(Ya.shape, dtype=Ya.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 50))
+    e_s = [mk() for _ in range(e2e_steps)]
+    e_e = [mk() for _ in range(e2e_steps)]
+    for _ in range(3):
+        X.copy_(Xh, non_blocking=True)
+        step()
+        Yh.copy_(Y, non_blocking=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        X.copy_(Xh, non_blocking=True)
+        Xa.copy_(Xah, non_blocking=True)
+        step()
+        Y_host = Yh.copy_(Y, non_blocking=True)
+        Yah.copy_(Ya, non_blocking=True)
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / e2e_steps
+    del Y_host
+
+    # ------------------------------------------------- max over ranks
+    t = torch.tensor([step_ms / args.steps, e2e_ms, k2_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step, ms_e2e, ms_k2 = (float(v) for v in t.cpu())
+
+    # ------------------------------------------------- context: cuBLAS bf16
+    cublas_tflops = None
+    if rank == 0:
+        A = torch.randn((M, K), dtype=torch.bfloat16, device=dev)
+        B = torch.randn((N, K), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            torch.matmul(A, B.T)
+        e0, e1 = mk(), mk()
+        e0.record(stream)
+        for _ in range(20):
+            torch.matmul(A, B.T)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cublas_tflops = 2.0 * M * N * K / (e0.elapsed_time(e1) / 20 * 1e-3) / 1e12
+        del A, B
+
+    # ------------------------------------------------- CPU baseline (oracle)
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
+        host = oracle_inputs_from_device({"svdq": svdq_w, "x_bits": x_bits, "bias_bits": d["bias"],
+                                          "xa_bits": da["X"], "awq_plain": awq_plain_host(da["W"])})
+        flops, secs, reps = time_oracle(host, args.cpu_budget, 8, 1152, 1152)
+        cpu = {"value": flops / secs / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{reps} x ({sample_text(8, 1152, 1152)}), {secs:.1f} s"}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    peaks = measured_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    k2_flops = 2.0 * M * N * K
+    achieved = k2_flops / (ms_k2 * 1e-3) / 1e12
+    value = step_flops() * world / (ms_step * 1e-3) / 1e12
+    traffic = recorded_traffic("w4a4_nvfp4_gemm_kernel")
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3, f32 accumulate)", "data": "synthetic",
+        "config": config_block(world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp4_peak, "traffic": traffic,
+                     "kernel": "w4a4_nvfp4_gemm_kernel",
+                     "peak_note": f"{peaks['source']} bf16 sustained x {FP4_OVER_BF16:g} "
+                                  f"(nominal FP4/BF16); vs nominal 9 PFLOP/s: {achieved / 9000:.3f}"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": step_flops() * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": X.numel() * 2 + Xa.numel() * 2,
+                "d2h_bytes_per_step": Y.numel() * 2 + Ya.numel() * 2, "ms_per_step": ms_e2e},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "kernels": {
+            "svdq_quantize_act_us": k1_ms * 1e3,
+            "svdq_quantize_act_gbs": quantize_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9,
+            "svdq_w4a4_linear_us": k2_ms * 1e3,
+            "svdq_w4a4_linear_tflops_4bit": achieved,
+            "svdq_w4a4_linear_tflops_incl_lowrank": layer_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12,
+            "layer_tflops": k2_flops / ((k1_ms + k2_ms) * 1e-3) / 1e12,
+            "awq_w4a16_linear_us": k3_ms * 1e3,
+            "awq_w4a16_linear_gbs": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / (k3_ms * 1e-3) / 1e9,
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "cublas_bf16_tflops_same_shape": cublas_tflops,
+        },
+        "device_status": status,
+    }
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

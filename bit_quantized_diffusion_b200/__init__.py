@@ -58,16 +58,17 @@ def awq_sz_bytes(Nrows: int, K: int) -> int:
     return N.load().awq_sz_bytes(Nrows, K)
 
 
-def svdq_quantize_act(X: torch.Tensor, L1t: torch.Tensor | None = None,
+def svdq_quantize_act(X: torch.Tensor, L1s: torch.Tensor | None = None,
                       smooth_inv: torch.Tensor | None = None, fmt="nvfp4",
                       codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
                       xl1: torch.Tensor | None = None, stream=None):
-    """Steps a1..a4 on X [M, K] bf16. Returns (codes, scales, xl1 or None)."""
+    """Steps a1..a4 on X [M, K] bf16. L1s is the [2, r, K] bf16 operand from
+    svdq_pack_lowrank. Returns (codes, scales, xl1 or None)."""
     lib = N.load()
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bf16 tensor")
     M, K = X.shape
-    r = 0 if L1t is None else L1t.shape[0]
+    r = 0 if L1s is None else L1s.shape[1]
     f = _fmt(fmt)
     dev = X.device
     if codes is None:
@@ -78,16 +79,32 @@ def svdq_quantize_act(X: torch.Tensor, L1t: torch.Tensor | None = None,
         xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
     _need(codes, lib.svdq_codes_bytes(f, M, K), "codes")
     _need(scales, lib.svdq_scales_bytes(f, M, K), "scales")
-    if L1t is not None and (L1t.dtype != torch.bfloat16 or tuple(L1t.shape) != (r, K)):
-        raise ValueError("L1t must be bf16 [r, K]")
+    if L1s is not None and (L1s.dtype != torch.bfloat16 or tuple(L1s.shape) != (2, r, K)):
+        raise ValueError("L1s must be bf16 [2, r, K]")
     if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
         raise ValueError("smooth_inv must be float32 [K]")
     if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < M * r):
         raise ValueError("xl1 must be float32 [M, r]")
-    N.check(lib.svdq_quantize_act(f, M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(L1t),
+    N.check(lib.svdq_quantize_act(f, M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(L1s),
                                   _ptr(codes), _ptr(scales), _ptr(xl1) if r else None,
                                   _stream(stream)), "svdq_quantize_act")
     return codes, scales, (xl1 if r else None)
+
+
+def svdq_pack_lowrank(L1: torch.Tensor, smooth_inv: torch.Tensor | None = None,
+                      L1s: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """L1 [K, r] bf16 (+ smooth_inv [K] f32) -> the [2, r, K] bf16 down-projection operand."""
+    lib = N.load()
+    if L1.dtype != torch.bfloat16 or L1.dim() != 2:
+        raise ValueError("L1 must be a 2-D bf16 tensor [K, r]")
+    K, r = L1.shape
+    if L1s is None:
+        L1s = torch.empty((2, r, K), dtype=torch.bfloat16, device=L1.device)
+    if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
+        raise ValueError("smooth_inv must be float32 [K]")
+    N.check(lib.svdq_pack_lowrank(K, r, _ptr(L1), _ptr(smooth_inv), _ptr(L1s), _stream(stream)),
+            "svdq_pack_lowrank")
+    return L1s
 
 
 def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int, N_: int,

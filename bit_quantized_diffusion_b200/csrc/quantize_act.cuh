@@ -1,22 +1,26 @@
 // quantize_act.cuh -- steps a1..a4 of the SVDQuant layer in one pass over X:
 // smoothing, group scale, 4-bit quantization + packing, and the rank-r
-// down-projection x_hat @ L1 on the tensor cores (Nunchaku README, "Engine
-// design" (b): the down projection and the quantizer share their input).
+// down-projection on the tensor cores (Nunchaku README, "Engine design" (b):
+// the down projection and the quantizer share their input).
+//
+// The down-projection reads the raw bf16 X tile that TMA brought in for the
+// quantizer: x_hat L1 = X (diag(smooth_inv) L1), and the smoothed factor
+// L1s = diag(smooth_inv) L1 comes pre-split into two bf16 planes (hi + lo, see
+// svdq_pack_lowrank), so two kind::f16 MMAs per K step give the product to
+// about 2^-17 relative, accumulated in float32 in tensor memory. The quantizer
+// threads therefore only read X and write codes and scales.
 //
 // One CTA owns 128 rows and a contiguous range of 64-column chunks of X. A
 // cluster of `ksplit` CTAs covers all of K for the same 128 rows; their partial
-// x_hat @ L1 sums are added through distributed shared memory in a fixed order.
+// sums are added through distributed shared memory in a fixed order.
 //
 // Warp roles (18 warps):
-//   warp 0      TMA producer: X chunk [128 x 64] bf16 and L1^T chunk [r x 64] bf16,
-//               both 128-byte swizzled, into a ring of stages
+//   warp 0      TMA producer: X chunk [128 x 64] bf16 (128-byte swizzle), the L1s
+//               hi and lo chunks [r x 64] bf16, and 64 smooth_inv values
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
 //   warps 2..17 quantizers; warp q handles rows 8q..8q+7, lane l handles row
-//               8q + l%8 and columns 16(l/8)..16(l/8)+15 of the chunk, i.e.
-//               exactly one NVFP4 group (a quarter of an INT4 group)
-// The quantizers also write x_hat split into bf16 hi + lo (no-swizzle K-major
-// core-matrix layout) for two tcgen05 kind::f16 MMAs per K step into one f32
-// accumulator in tensor memory.
+//               8q + l%8 and columns 16(l/8)..16(l/8)+15 of the chunk: exactly one
+//               NVFP4 group (a quarter of an INT4 group)
 #pragma once
 
 #include "sm100.cuh"
@@ -26,9 +30,9 @@ namespace svdq {
 constexpr int kQaWarps = 18;
 constexpr int kQaThreads = kQaWarps * 32;
 constexpr int kQaQuantWarps = 16;
-constexpr int kQaChunk = 64;                   // columns per stage
+constexpr int kQaChunk = 64;                        // columns per stage
 constexpr int kQaXStageBytes = 128 * kQaChunk * 2;  // 16 KB
-constexpr int kQaATileBytes = 128 * kQaChunk * 2;   // one bf16 [128 x 64] tile
+constexpr int kQaSmoothBytes = kQaChunk * 4;        // 256 B
 
 struct QuantActParams {
   int M, K, r;
@@ -44,17 +48,18 @@ struct QuantActParams {
 
 struct QaSmem {
   // byte offsets from the 1024-aligned dynamic shared memory base
-  uint32_t ring, stage_bytes, a_tiles, bars, tmem_slot;
+  uint32_t ring, stage_bytes, l1_off, sm_off, table, bars, tmem_slot;
 };
 
 __host__ __device__ inline QaSmem qa_smem_layout(int r, int stages) {
   QaSmem s;
   s.ring = 0;
-  s.stage_bytes = kQaXStageBytes + r * 128;
-  s.a_tiles = s.ring + stages * s.stage_bytes;
-  const uint32_t a_bytes = r > 0 ? 4 * kQaATileBytes : 0;  // 2 buffers x (hi, lo)
-  s.bars = s.a_tiles + a_bytes;
-  s.tmem_slot = s.bars + 8 * (2 * stages + 5);
+  s.l1_off = kQaXStageBytes;                       // hi plane, then lo plane
+  s.sm_off = kQaXStageBytes + 2 * r * 128;         // smooth_inv chunk
+  s.stage_bytes = (s.sm_off + kQaSmoothBytes + 1023) / 1024 * 1024;
+  s.table = s.ring + stages * s.stage_bytes;       // E4M3 (value, reciprocal) x 128
+  s.bars = s.table + 128 * 8;
+  s.tmem_slot = s.bars + 8 * (2 * stages + 1);
   return s;
 }
 
@@ -75,6 +80,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int NS = p.stages;
   const int r = p.r;
+  const bool smoothing = p.smooth_inv != nullptr;
 
   const int ks = blockIdx.x % p.ksplit;
   const int rb = blockIdx.y;
@@ -85,30 +91,28 @@ __global__ void __launch_bounds__(kQaThreads, 1)
 
   auto bar_full = [&](int s) { return sbase + L.bars + 8 * s; };
   auto bar_empty = [&](int s) { return sbase + L.bars + 8 * (NS + s); };
-  auto bar_afull = [&](int a) { return sbase + L.bars + 8 * (2 * NS + a); };
-  auto bar_aempty = [&](int a) { return sbase + L.bars + 8 * (2 * NS + 2 + a); };
-  const uint32_t bar_acc = sbase + L.bars + 8 * (2 * NS + 4);
+  const uint32_t bar_acc = sbase + L.bars + 8 * (2 * NS);
   auto x_stage = [&](int s) { return sbase + L.ring + s * L.stage_bytes; };
-  auto l1_stage = [&](int s) { return x_stage(s) + kQaXStageBytes; };
-  auto a_hi = [&](int a) { return sbase + L.a_tiles + a * 2 * kQaATileBytes; };
-  auto a_lo = [&](int a) { return a_hi(a) + kQaATileBytes; };
-
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
   const uint32_t tmem_cols = r <= 32 ? 32 : (r <= 64 ? 64 : (r <= 128 ? 128 : 256));
+  float2* table = reinterpret_cast<float2*>(smem + L.table);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), r > 0 ? 1 : kQaQuantWarps);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(bar_afull(a), kQaQuantWarps);
-      mbar_init(bar_aempty(a), 1);
+      // the quantizer warps finish reading X, and the MMAs finish reading X and L1s
+      mbar_init(bar_empty(s), kQaQuantWarps + (r > 0 ? 1 : 0));
     }
     mbar_init(bar_acc, 1);
     fence_barrier_init();
     prefetch_tmap(&tm_x);
     if (r > 0) prefetch_tmap(&tm_l1);
+  }
+  if (kFmt == 0 && threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
+    // every E4M3 scale code: its value and correctly rounded float32 reciprocal
+    const uint32_t c = threadIdx.x - 64;
+    const float v = c < 0x7F ? e4m3_value(c) : 0.0f;
+    table[c] = make_float2(v, v != 0.0f ? __frcp_rn(v) : 0.0f);
   }
   if (warp == 1 && r > 0) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
@@ -122,39 +126,42 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (elect_one()) {
-      const uint32_t tx = kQaXStageBytes + r * 128;
+      const uint32_t tx = kQaXStageBytes + 2 * r * 128 + (smoothing ? kQaSmoothBytes : 0);
       for (int i = 0; i < nchunks; ++i) {
         const int s = i % NS;
         if (!mbar_wait(bar_empty(s), ((i / NS) & 1) ^ 1, p.status)) break;
+        const int kc = kc0 + i;
         mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(x_stage(s), &tm_x, bar_full(s), (kc0 + i) * kQaChunk, rb * 128);
-        if (r > 0) tma_load_2d(l1_stage(s), &tm_l1, bar_full(s), (kc0 + i) * kQaChunk, 0);
+        tma_load_2d(x_stage(s), &tm_x, bar_full(s), kc * kQaChunk, rb * 128);
+        if (r > 0) {
+          tma_load_2d(x_stage(s) + L.l1_off, &tm_l1, bar_full(s), kc * kQaChunk, 0);
+          tma_load_2d(x_stage(s) + L.l1_off + r * 128, &tm_l1, bar_full(s), kc * kQaChunk, r);
+        }
+        if (smoothing)
+          bulk_load(x_stage(s) + L.sm_off, p.smooth_inv + kc * kQaChunk, kQaSmoothBytes,
+                    bar_full(s));
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (r > 0 && elect_one()) {
       const uint32_t idesc = idesc_bf16_f32(128, r, false, false);
-      bool ok = true;
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const int s = i % NS, a = i & 1;
-        ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status) &&
-             mbar_wait(bar_afull(a), (i >> 1) & 1, p.status);
-        if (!ok) break;
+      for (int i = 0; i < nchunks; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(bar_full(s), (i / NS) & 1, p.status)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kQaChunk / 16; ++kk) {
-          // A: no-swizzle K-major, core matrices 8 rows x 16 B; K-adjacent ones
-          // 128 B apart (LBO), 8-row groups 1024 B apart (SBO); 16 K = 256 B.
-          const uint64_t ah = smem_desc(a_hi(a) + kk * 256, 128, 1024, kSwizzleNone);
-          const uint64_t al = smem_desc(a_lo(a) + kk * 256, 128, 1024, kSwizzleNone);
-          // B: L1^T rows (r of them), 128 B each, 128-byte swizzle; 16 K = 32 B.
-          const uint64_t bd = smem_desc(l1_stage(s) + kk * 32, 16, 1024, kSwizzle128B);
-          mma_f16(tmem_base, ah, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_f16(tmem_base, al, bd, idesc, 1u);
+          // A: the X tile, 128 rows x 128 B, 128-byte swizzle; 16 K = 32 B
+          const uint64_t ad = smem_desc(x_stage(s) + kk * 32, 16, 1024, kSwizzle128B);
+          // B: L1s hi / lo planes, r rows x 128 B each, 128-byte swizzle
+          const uint64_t bh = smem_desc(x_stage(s) + L.l1_off + kk * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bl =
+              smem_desc(x_stage(s) + L.l1_off + r * 128 + kk * 32, 16, 1024, kSwizzle128B);
+          mma_f16(tmem_base, ad, bh, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_f16(tmem_base, ad, bl, idesc, 1u);
         }
         tc_commit(bar_empty(s));
-        tc_commit(bar_aempty(a));
       }
       tc_commit(bar_acc);
     }
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       const int kc = kc0 + i;
       ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status);
       if (!ok) break;
-      // -- load 16 bf16 of this row from the 128B-swizzled X tile
+      // -- 16 bf16 of this row from the 128B-swizzled X tile
       float xh[16];
       {
         const uint32_t rowbase = x_stage(s) + row * 128;
@@ -190,18 +197,22 @@ __global__ void __launch_bounds__(kQaThreads, 1)
           }
         }
       }
-      // -- a1: smoothing, one float32 multiply
-      if (p.smooth_inv != nullptr) {
-        const float4* sp = reinterpret_cast<const float4*>(p.smooth_inv + kc * kQaChunk + 16 * q);
+      // -- a1: smoothing, one float32 multiply per element
+      if (smoothing) {
+        const float4* sp = reinterpret_cast<const float4*>(smem + (x_stage(s) - sbase) + L.sm_off) +
+                           4 * q;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float4 sv = __ldg(sp + j);
+          const float4 sv = sp[j];
           xh[4 * j + 0] = __fmul_rn(xh[4 * j + 0], sv.x);
           xh[4 * j + 1] = __fmul_rn(xh[4 * j + 1], sv.y);
           xh[4 * j + 2] = __fmul_rn(xh[4 * j + 2], sv.z);
           xh[4 * j + 3] = __fmul_rn(xh[4 * j + 3], sv.w);
         }
       }
+      // this warp no longer reads the stage's shared memory
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(s));
       // -- a2 + a3: group scale and codes
       float amax = 0.0f;
 #pragma unroll
@@ -209,18 +220,16 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       uint32_t code_lo = 0, code_hi = 0;
       if (kFmt == 0) {
         const uint32_t sc = e4m3_code(__fdiv_rn(amax, 6.0f));
-        const float sval = e4m3_value(sc);
-        if (sval != 0.0f) {
-          const float rcp = __frcp_rn(sval);
-          float y0[8], y1[8];
+        const float2 vr = table[sc];  // (decoded scale, its reciprocal)
+        float y0[8], y1[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            y0[j] = __fmul_rn(xh[j], rcp);
-            y1[j] = __fmul_rn(xh[8 + j], rcp);
-          }
-          code_lo = e2m1x8(y0);
-          code_hi = e2m1x8(y1);
+        for (int j = 0; j < 8; ++j) {
+          y0[j] = __fmul_rn(xh[j], vr.y);
+          y1[j] = __fmul_rn(xh[8 + j], vr.y);
         }
+        const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
+        code_lo = live ? e2m1x8(y0) : 0u;
+        code_hi = live ? e2m1x8(y1) : 0u;
         // gather the row's four scale bytes into one word (lanes l, l+8, l+16, l+24)
         const uint32_t b1 = __shfl_down_sync(0xffffffffu, sc, 8);
         const uint32_t b2 = __shfl_down_sync(0xffffffffu, sc, 16);
@@ -255,43 +264,14 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + q * 8) =
             make_uint2(code_lo, code_hi);
       }
-      // -- a4 operand: x_hat as bf16 hi + lo for the tensor cores
-      if (r > 0) {
-        const int a = i & 1;
-        ok = mbar_wait(bar_aempty(a), ((i >> 1) & 1) ^ 1, p.status);
-        if (!ok) break;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float x0 = xh[8 * h + 2 * j], x1 = xh[8 * h + 2 * j + 1];
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(hb);
-            const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-            hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
-            lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
-          }
-          const uint32_t off = (row >> 3) * 1024 + (2 * q + h) * 128 + (row & 7) * 16;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi(a) + off), "r"(hi[0]),
-                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
-                       : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo(a) + off), "r"(lo[0]),
-                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
-                       : "memory");
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_afull(a));
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty(s));
-      }
     }
     // ------------------------------------------------------------ xl1 epilogue
+    // The reduction buffer reuses the ring: every quantizer warp must be done
+    // reading X before any of them writes partial sums there.
+    if (r > 0 && p.ksplit > 1) asm volatile("bar.sync 1, %0;" ::"n"(kQaQuantWarps * 32) : "memory");
     if (r > 0 && ok && mbar_wait(bar_acc, 0, p.status)) {
       tc_fence_after();
-      const int quad = warp & 3;        // tensor-memory lanes this warp may read
+      const int quad = warp & 3;         // tensor-memory lanes this warp may read
       const int part = (warp - 2) >> 2;  // which quarter of the r columns
       const int trow = quad * 32 + lane;
       const int ncol = r / 4, c_begin = part * ncol;
@@ -347,6 +327,23 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   if (warp == 1 && r > 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// L1s = diag(smooth_inv) L1 as two bf16 planes [2][r][K] (hi, lo): hi = RN_bf16(v),
+// lo = RN_bf16(v - hi), v = RN32(smooth_inv[k] * L1[k][j]).
+__global__ void pack_lowrank_kernel(const __nv_bfloat16* L1, const float* smooth_inv,
+                                    __nv_bfloat16* L1s, int K, int r) {
+  const size_t total = static_cast<size_t>(K) * r;
+  for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(t / K), k = static_cast<int>(t % K);
+    float v = __bfloat162float(L1[static_cast<size_t>(k) * r + j]);
+    if (smooth_inv != nullptr) v = __fmul_rn(v, smooth_inv[k]);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+    L1s[t] = hi;
+    L1s[total + t] = lo;
   }
 }
 

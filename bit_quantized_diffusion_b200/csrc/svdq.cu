@@ -143,14 +143,14 @@ size_t awq_sz_bytes(int N, int K) {
 }
 
 svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
-                              const float* smooth_inv, const void* L1t, void* codes,
+                              const float* smooth_inv, const void* L1s, void* codes,
                               void* scales, float* xl1, svdq_stream_t stream) {
   if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || K < 64 || K % 64 || !rank_ok(r) || ldx < K) return SVDQ_ERR_INVALID_ARG;
   if (X == nullptr || codes == nullptr || scales == nullptr) return SVDQ_ERR_INVALID_ARG;
-  if ((r > 0) != (L1t != nullptr) || (r > 0) != (xl1 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1s != nullptr) || (r > 0) != (xl1 != nullptr)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || ldx % 8 ||
-      (smooth_inv && !aligned16(smooth_inv)) || (L1t && !aligned16(L1t)) ||
+      (smooth_inv && !aligned16(smooth_inv)) || (L1s && !aligned16(L1s)) ||
       (xl1 && !aligned16(xl1)))
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
@@ -161,7 +161,7 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
-    if (!make_tmap_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, K, r,
+    if (!make_tmap_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1s, K, 2 * r,
                       static_cast<uint64_t>(K) * 2, 64, r, CU_TENSOR_MAP_SWIZZLE_128B))
       return SVDQ_ERR_CUDA;
   } else {
@@ -173,8 +173,9 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   int ksplit = 1;
   while (ksplit * 2 <= 8 && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= d->num_sms)
     ksplit *= 2;
-  const int stage_bytes = kQaXStageBytes + r * 128;
-  const int avail = 232448 - 1024 - 256 - (r > 0 ? 4 * kQaATileBytes : 0);
+  const QaSmem lay = qa_smem_layout(r, 1);
+  const int stage_bytes = static_cast<int>(lay.stage_bytes);
+  const int avail = 232448 - 1024 - 1024 - 512;
   int stages = avail / stage_bytes;
   if (stages > 8) stages = 8;
   if (stages < 2) return SVDQ_ERR_UNSUPPORTED;
@@ -261,7 +262,9 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.ldy = ldy;
   p.out_f32 = out == SVDQ_OUT_F32;
   p.status = d->status;
-  dim3 grid((M + kGmBM - 1) / kGmBM, (N + kGmBN - 1) / kGmBN, 1);
+  p.tiles_m = (M + kGmBM - 1) / kGmBM;
+  p.tiles = p.tiles_m * ((N + kGmBN - 1) / kGmBN);
+  const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
   w4a4_nvfp4_gemm_kernel<<<grid, kGmThreads, kGmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       tm_a, tm_b, tm_l2, p);
   return launch_status();
@@ -287,7 +290,7 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   const int nblocks = (N + 15) / 16;
-  dim3 grid((nblocks + 3) / 4);
+  dim3 grid((nblocks + kAwqBlocksPerCta - 1) / kAwqBlocksPerCta);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch ((M + 7) / 8) {
     case 1: awq_gemv_kernel<1><<<grid, kAwqThreads, 0, s>>>(p); break;
@@ -404,6 +407,19 @@ svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K
     return launch_status();
   }
   return SVDQ_ERR_INVALID_ARG;
+}
+
+svdq_status svdq_pack_lowrank(int K, int r, const void* L1, const float* smooth_inv, void* L1s,
+                              svdq_stream_t stream) {
+  if (K < 64 || K % 64 || r < 16 || r > 256 || r % 16 || !L1 || !L1s) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(L1) || !aligned16(L1s) || (smooth_inv && !aligned16(smooth_inv)))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const size_t n = static_cast<size_t>(K) * r;
+  pack_lowrank_kernel<<<grid_for(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(L1), smooth_inv, static_cast<__nv_bfloat16*>(L1s), K, r);
+  return launch_status();
 }
 
 svdq_status svdq_check_device_status(svdq_stream_t stream) {

@@ -1,0 +1,52 @@
+"""User-facing layers over the C ABI: the SVDQ W4A4 linear and the AWQ W4A16
+linear (the ``SVDQW4A4Linear`` / ``AWQW4A16Linear`` runtime layers of the
+Diffusers blog, "quantization_config"), with preallocated workspaces so a
+forward call is two (or one) library calls and no allocation."""
+
+from __future__ import annotations
+
+import torch
+
+from . import awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_scales_bytes, svdq_w4a4_linear
+
+
+class SvdqW4A4Linear:
+    """Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + bias on prepared weights."""
+
+    def __init__(self, weights: dict, bias: torch.Tensor | None, max_tokens: int):
+        self.w = weights
+        self.bias = bias
+        self.fmt = weights["fmt"]
+        self.N, self.K, self.r = weights["N"], weights["K"], weights["r"]
+        dev = weights["w_codes"].device
+        self.max_tokens = max_tokens
+        self.codes = torch.empty(svdq_codes_bytes(self.fmt, max_tokens, self.K), dtype=torch.uint8,
+                                 device=dev)
+        self.scales = torch.empty(svdq_scales_bytes(self.fmt, max_tokens, self.K), dtype=torch.uint8,
+                                  device=dev)
+        self.xl1 = torch.empty((max_tokens, self.r), dtype=torch.float32, device=dev) if self.r else None
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        M = x.shape[0]
+        if M > self.max_tokens:
+            raise ValueError(f"{M} tokens > workspace for {self.max_tokens}")
+        xl1 = self.xl1[:M] if self.r else None
+        codes, scales, xl1 = svdq_quantize_act(x, self.w["L1s"], self.w["smooth_inv"], fmt=self.fmt,
+                                               codes=self.codes, scales=self.scales, xl1=xl1,
+                                               stream=stream)
+        return svdq_w4a4_linear(codes, scales, xl1, self.w["w_codes"], self.w["w_scales"], self.w["L2"],
+                                self.bias, M, self.N, self.K, fmt=self.fmt, Y=y, stream=stream)
+
+    __call__ = forward
+
+
+class AwqW4A16Linear:
+    def __init__(self, weights: dict, bias: torch.Tensor | None):
+        self.w = weights
+        self.bias = bias
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        return awq_w4a16_linear(x, self.w["qweight"], self.w["sz"], self.bias, self.w["N"], Y=y,
+                                stream=stream)
+
+    __call__ = forward

@@ -98,17 +98,19 @@ size_t awq_sz_bytes(int N, int K);
  *
  * X          device, bf16 [M, ldx] (first K columns used), ldx % 8 == 0
  * smooth_inv device, float32 [K], or NULL
- * L1t        device, bf16 [r, K]: L1 stored transposed (K contiguous); NULL iff r == 0
+ * L1s        device, the down-projection operand from svdq_pack_lowrank: bf16
+ *            [2][r][K] = diag(smooth_inv) L1, transposed, as hi and lo planes;
+ *            NULL iff r == 0
  * codes      device, svdq_codes_bytes(format, M, K) bytes, written
  * scales     device, svdq_scales_bytes(format, M, K) bytes, written (padding rows too)
  * xl1        device, float32 [M, r], written; NULL iff r == 0
  * Codes and scales are bit-exact functions of the inputs. xl1 is computed on the
- * tensor cores with x_hat split into two bf16 terms (hi + lo) and float32
- * accumulation. This call also serves as the weight quantizer (residual R given
- * as bf16, smooth_inv NULL, r 0).
+ * tensor cores as X (hi + lo) with float32 accumulation, which equals x_hat L1 to
+ * about 2^-17 relative per term. This call also serves as the weight quantizer
+ * (residual R given as bf16, smooth_inv NULL, r 0).
  */
 svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
-                              const float* smooth_inv, const void* L1t, void* codes,
+                              const float* smooth_inv, const void* L1s, void* codes,
                               void* scales, float* xl1, svdq_stream_t stream);
 
 /*
@@ -174,6 +176,21 @@ svdq_status svdq_pack(svdq_pack_kind kind, svdq_format format, int rows, int K,
 svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K,
                         const void* tiled_codes, const void* tiled_scales, void* plain_codes,
                         void* plain_scales, void* plain_zeros, svdq_stream_t stream);
+
+/*
+ * svdq_pack_lowrank -- the down-projection operand of svdq_quantize_act. The
+ * smoothing folds into the factor (x_hat L1 = X diag(smooth_inv) L1), which is
+ * split into two bf16 terms so the tensor cores see it at about 16-bit-squared
+ * precision:
+ *   v = RN32(smooth_inv[k] * L1[k][j]),  hi = RN_bf16(v),  lo = RN_bf16(v - hi)
+ *   L1s[0][j][k] = hi, L1s[1][j][k] = lo
+ * L1          device, bf16 [K, r] (the SVD factor, K rows)
+ * smooth_inv  device, float32 [K] or NULL (then v = L1)
+ * L1s         device, bf16 [2][r][K], written
+ * K % 64 == 0, r % 16 == 0, 16 <= r <= 256.
+ */
+svdq_status svdq_pack_lowrank(int K, int r, const void* L1, const float* smooth_inv, void* L1s,
+                              svdq_stream_t stream);
 
 /*
  * svdq_check_device_status -- synchronises `stream`, then reads and clears the

@@ -30,6 +30,10 @@ AWQ qweight, MMA-fragment order
     (row offsets within the block, column offsets from 64 g + 16 j).
     Byte offset of w_j: ((b * (K // 64) + g) * 32 + t) * 16 + 4 j.
 
+Down-projection operand L1s (the smoothing folded into the factor)
+    v = RN32(smooth_inv[k] * L1[k, j]), hi = BF16(v), lo = BF16(RN32(v - hi));
+    planes [2][r][K]: L1s[0, j, k] = hi, L1s[1, j, k] = lo.
+
 AWQ scales and zeros, interleaved
     bf16 pairs (s, z) at [N / 16][K // 64][16 rows][2], rows padded with (0, 0).
 """
@@ -158,3 +162,15 @@ def untile_awq_sz(tiled: np.ndarray, N: int, K: int):
     s = t[..., 0].transpose(0, 2, 1).reshape(Np, G)[:N]
     z = t[..., 1].transpose(0, 2, 1).reshape(Np, G)[:N]
     return s.copy(), z.copy()
+
+
+# ------------------------------------------------------ down-projection operand
+def lowrank_operand(L1: np.ndarray, smooth_inv: np.ndarray | None) -> np.ndarray:
+    """L1 [K, r] (bf16 values), smooth_inv [K] (float32 values) -> [2, r, K] bf16 values."""
+    from .formats import bf16_round, rn32
+    v = np.asarray(L1, np.float64).T.copy()
+    if smooth_inv is not None:
+        v = rn32(v * np.asarray(smooth_inv, np.float64)[None, :])
+    hi = bf16_round(v)
+    lo = bf16_round(rn32(v - hi))
+    return np.stack([hi, lo])

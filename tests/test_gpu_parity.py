@@ -35,6 +35,9 @@ SMALL = [
     WL.custom_svdq("one_row", 1, 128, 48, 16, seed=13),
     WL.custom_svdq("r0", 130, 256, 160, 0, seed=14),
     WL.custom_svdq("r256", 200, 512, 256, 256, seed=15, spike_rank=8, spike_sv=5.0),
+    # more tiles than SMs: every persistent CTA walks several tiles, both accumulators
+    WL.custom_svdq("many_tiles", 2048, 512, 2816, 32, seed=18),
+    WL.custom_svdq("many_tiles_r128", 2176, 256, 2560, 128, seed=19),
 ]
 
 
@@ -42,8 +45,8 @@ def _quantize_gpu(bq, layer, X_bits, fmt, with_lowrank=True, smooth=True):
     X = C.bf16_tensor(X_bits)
     si = C.f32_tensor(layer["smooth_inv"]) if smooth else None
     r = layer["L1"].shape[1] if with_lowrank else 0
-    L1t = C.bf16_tensor(F.bf16_bits(layer["L1"].T.copy())) if r else None
-    codes, scales, xl1 = bq.svdq_quantize_act(X, L1t, si, fmt=fmt)
+    L1s = C.bf16_tensor(F.bf16_bits(LO.lowrank_operand(layer["L1"], layer["smooth_inv"] if smooth else None))) if r else None
+    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si, fmt=fmt)
     assert bq.svdq_check_device_status() == 0
     return codes.cpu().numpy(), scales.cpu().numpy(), (xl1.cpu().numpy() if xl1 is not None else None)
 
@@ -162,14 +165,26 @@ def test_end_to_end_layer(bq):
     fwd = S.svdq_forward("nvfp4", layer["x_bits"], layer["smooth_inv"], layer["L1"], layer["L2"],
                          layer["w_codes"], layer["w_scales"], layer["bias_bits"])
     X = C.bf16_tensor(layer["x_bits"])
-    L1t = C.bf16_tensor(F.bf16_bits(layer["L1"].T.copy()))
-    codes, scales, xl1 = bq.svdq_quantize_act(X, L1t, C.f32_tensor(layer["smooth_inv"]))
+    si = C.f32_tensor(layer["smooth_inv"])
+    L1s = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si)
+    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si)
     y = bq.svdq_w4a4_linear(codes, scales, xl1, C.u8_tensor(S.pack_nibbles(layer["w_codes"]).reshape(-1)),
                             C.u8_tensor(LO.tile_nvfp4_scales(layer["w_scales"])),
                             C.bf16_tensor(F.bf16_bits(layer["L2"])), C.bf16_tensor(layer["bias_bits"]),
                             M=shape.M, N_=shape.N, K=shape.K)
     assert bq.svdq_check_device_status() == 0
     C.assert_gemm_close(y.float().cpu().numpy().astype(np.float64), fwd["Y"], bf16_out=True)
+
+
+@pytest.mark.parametrize("r,with_smooth", [(16, True), (32, True), (128, False), (256, True)])
+def test_pack_lowrank_matches_oracle(bq, r, with_smooth):
+    rng = np.random.default_rng(40 + r)
+    K = 320
+    L1 = F.bf16_round(rng.standard_normal((K, r)) * 0.3)
+    si = F.rn32(rng.uniform(0.05, 4.0, K)) if with_smooth else None
+    got = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(L1)), C.f32_tensor(si) if with_smooth else None)
+    want = F.bf16_bits(LO.lowrank_operand(L1, si))
+    assert np.array_equal(C.bf16_bits_of(got), want)
 
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
@@ -248,3 +263,35 @@ def test_timeout_path_reports_and_recovers(bq):
     codes, scales, _ = bq.svdq_quantize_act(x, None, None)
     assert bq.svdq_check_device_status() == 0
     assert not codes.any() and not scales.any()
+
+
+@pytest.mark.slow
+def test_full_size_qkv_sampled(bq):
+    """The FLUX-like QKV workload at full size, in the launch configuration the
+    benchmark times: all codes and scales bit-exact, xl1 and Y on sampled rows."""
+    shape = WL.QKV
+    layer = C.oracle_layer(shape)
+    x = F.bf16_from_bits(layer["x_bits"])
+    X = C.bf16_tensor(layer["x_bits"])
+    si = C.f32_tensor(layer["smooth_inv"])
+    L1s = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si)
+    wc, ws, _ = bq.svdq_quantize_act(C.bf16_tensor(F.bf16_bits(layer["R"])), None, None)
+    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si)
+    y = bq.svdq_w4a4_linear(codes, scales, xl1, wc, ws, C.bf16_tensor(F.bf16_bits(layer["L2"])),
+                            C.bf16_tensor(layer["bias_bits"]), M=shape.M, N_=shape.N, K=shape.K)
+    assert bq.svdq_check_device_status() == 0
+    assert np.array_equal(wc.cpu().numpy(), S.pack_nibbles(layer["w_codes"]).reshape(-1))
+    assert np.array_equal(ws.cpu().numpy(), LO.tile_nvfp4_scales(layer["w_scales"]))
+    xhat = S.smooth(x, layer["smooth_inv"])
+    q, sc = S.quantize_nvfp4(xhat)
+    assert np.array_equal(codes.cpu().numpy(), S.pack_nibbles(q).reshape(-1))
+    assert np.array_equal(scales.cpu().numpy(), LO.tile_nvfp4_scales(sc))
+    rows = np.unique(np.concatenate([np.arange(0, shape.M, 97), [shape.M - 1]]))
+    ref_xl1 = S.down_proj(xhat[rows], layer["L1"])
+    got_xl1 = xl1.cpu().numpy()[rows].astype(np.float64)
+    assert np.all(np.abs(got_xl1 - ref_xl1) <= C.xl1_bound(xhat[rows], layer["L1"]))
+    ref = S.w4a4_linear(S.dequant_nvfp4(q[rows], sc[rows]),
+                        S.dequant_nvfp4(layer["w_codes"], layer["w_scales"]),
+                        S.down_proj(xhat[rows], layer["L1"]), layer["L2"],
+                        F.bf16_from_bits(layer["bias_bits"]))
+    C.assert_gemm_close(y.float().cpu().numpy()[rows].astype(np.float64), ref, bf16_out=True)

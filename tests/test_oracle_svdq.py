@@ -254,3 +254,25 @@ def test_smoothing_is_one_float32_multiply():
     xh = S.smooth(x, si)
     assert xh[0, 0] == float(np.float32(1.0) * np.float32(1 / 3.0))
     assert xh[0, 1] == 1.5
+
+
+def test_lowrank_operand_split():
+    """hi + lo carries smooth_inv * L1 to about 2^-17 relative; both are bf16;
+    without smoothing the lo plane is zero. Summed, the split down-projection
+    X (hi + lo) equals x_hat L1 within that bound."""
+    rng = np.random.default_rng(14)
+    K, r = 128, 16
+    L1 = F.bf16_round(rng.standard_normal((K, r)))
+    si = F.rn32(rng.uniform(0.1, 3.0, K))
+    op = L.lowrank_operand(L1, si)
+    assert op.shape == (2, r, K)
+    assert np.array_equal(F.bf16_round(op), op)
+    v = F.rn32(L1.T * si[None, :])
+    assert np.all(np.abs(op[0] + op[1] - v) <= np.abs(v) * 2.0 ** -17)
+    plain = L.lowrank_operand(L1, None)
+    assert np.array_equal(plain[0], L1.T) and not plain[1].any()
+    x = F.bf16_round(rng.standard_normal((8, K)))
+    xhat = S.smooth(x, si)
+    ref = S.down_proj(xhat, L1)
+    got = x @ (op[0] + op[1]).T
+    assert np.all(np.abs(got - ref) <= (np.abs(xhat) @ np.abs(L1)) * 2.0 ** -16)
