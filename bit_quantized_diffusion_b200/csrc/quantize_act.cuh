@@ -69,7 +69,7 @@ __host__ inline size_t qa_smem_bytes(int r, int stages) {
 }
 
 template <int kFmt>  // 0: NVFP4 (E2M1, UE4M3 per 16), 1: INT4 (FP16 per 64)
-__global__ void __launch_bounds__(kQaThreads, 1)
+__global__ void __launch_bounds__(kQaThreads, 2)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_l1, const QuantActParams p) {
   extern __shared__ uint8_t smem_raw[];

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -65,6 +67,11 @@ svdq_status device_setup(DeviceInfo** out) {
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kGmSmemBytes)) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(awq_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     d.status = static_cast<uint32_t*>(st);
     d.ready = true;
@@ -170,17 +177,37 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
 
   const int row_blocks = (M + 127) / 128;
   const int kc_total = K / 64;
-  int ksplit = 1;
-  while (ksplit * 2 <= 8 && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= d->num_sms)
-    ksplit *= 2;
+  // Ring depth: two CTAs per SM when at least 3 stages fit in half the shared
+  // memory, else one CTA per SM with up to 8 stages.
   const QaSmem lay = qa_smem_layout(r, 1);
   const int stage_bytes = static_cast<int>(lay.stage_bytes);
-  const int avail = 232448 - 1024 - 1024 - 512;
-  int stages = avail / stage_bytes;
-  if (stages > 8) stages = 8;
-  if (stages < 2) return SVDQ_ERR_UNSUPPORTED;
-  // the ring is reused for the cross-CTA reduction of the [128 x r] partial sums
-  if (r > 0 && 128 * (r + 4) * 4 > stages * stage_bytes) return SVDQ_ERR_UNSUPPORTED;
+  const int fixed = static_cast<int>(qa_smem_bytes(r, 0));
+  const int red_bytes = r > 0 ? 128 * (r + 4) * 4 : 0;  // reduction buffer, reuses the ring
+  auto fits = [&](int st, int budget) {
+    return st >= 2 && fixed + st * stage_bytes <= budget && red_bytes <= st * stage_bytes;
+  };
+  int stages = 0, per_sm = 1;
+  const int half_budget = 113 * 1024, full_budget = 227 * 1024;
+  for (int st = 8; st >= 3; --st)
+    if (fits(st, half_budget)) { stages = st; per_sm = 2; break; }
+  if (stages == 0)
+    for (int st = 8; st >= 2; --st)
+      if (fits(st, full_budget)) { stages = st; break; }
+  if (stages == 0) return SVDQ_ERR_UNSUPPORTED;
+  const size_t smem_bytes = qa_smem_bytes(r, stages);
+  auto kern = format == SVDQ_NVFP4_G16 ? quantize_act_kernel<0> : quantize_act_kernel<1>;
+
+  // K split: the largest power of two (<= 8, <= 4 with two CTAs per SM so a
+  // cluster's CTAs fit in one GPC alongside others, <= K/64) whose CTAs fit in
+  // one wave of the SMs.
+  const int slots = per_sm * d->num_sms;
+  const int s_cap = per_sm == 2 ? 4 : 8;
+  int ksplit = 1;
+  while (ksplit * 2 <= s_cap && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= slots)
+    ksplit *= 2;
+  if (std::getenv("SVDQ_DEBUG") != nullptr)
+    std::fprintf(stderr, "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d\n",
+                 M, K, r, stages, per_sm, ksplit, ksplit * row_blocks);
 
   QuantActParams p;
   p.M = M;
@@ -198,7 +225,7 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ksplit, row_blocks, 1);
   cfg.blockDim = dim3(kQaThreads, 1, 1);
-  cfg.dynamicSmemBytes = qa_smem_bytes(r, stages);
+  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -207,9 +234,7 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (r > 0 && ksplit > 1) ? 1 : 0;
-  cudaError_t e = format == SVDQ_NVFP4_G16
-                      ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<0>, tm_x, tm_l1, p)
-                      : cudaLaunchKernelEx(&cfg, quantize_act_kernel<1>, tm_x, tm_l1, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l1, p);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
@@ -236,7 +261,7 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
 
-  CUtensorMap tm_a, tm_b, tm_l2;
+  CUtensorMap tm_a, tm_b, tm_l2, tm_y;
   if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, kGmBKBytes,
                     kGmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, kGmBKBytes,
@@ -249,6 +274,12 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   } else {
     tm_l2 = tm_a;
   }
+  // output: 32 x 32 boxes, bf16 rows of 64 B (64-byte swizzle) or f32 rows of 128 B
+  const bool f32 = out == SVDQ_OUT_F32;
+  if (!make_tmap_2d(&tm_y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    Y, N, M, static_cast<uint64_t>(ldy) * esz, 32, 32,
+                    f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ERR_CUDA;
   GemmParams p;
   p.M = M;
   p.N = N;
@@ -266,7 +297,7 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.tiles = p.tiles_m * ((N + kGmBN - 1) / kGmBN);
   const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
   w4a4_nvfp4_gemm_kernel<<<grid, kGmThreads, kGmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      tm_a, tm_b, tm_l2, p);
+      tm_a, tm_b, tm_l2, tm_y, p);
   return launch_status();
 }
 
@@ -280,27 +311,32 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
-  AwqParams p;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.X = static_cast<const __nv_bfloat16*>(X);
-  p.qweight = static_cast<const uint4*>(qweight);
-  p.sz = static_cast<const uint32_t*>(sz);
-  p.bias = static_cast<const __nv_bfloat16*>(bias);
-  p.Y = static_cast<__nv_bfloat16*>(Y);
+  // tokens per launch: at most 16 (two 8-token MMA blocks), and as many X rows
+  // as fit in shared memory beside the weight staging
+  const size_t smem_cap = 232448;
+  int mc = M < 16 ? M : 16;
+  while (mc > 1 && awq_smem_bytes(mc, K) > smem_cap) --mc;
+  if (awq_smem_bytes(mc, K) > smem_cap) return SVDQ_ERR_UNSUPPORTED;
   const int nblocks = (N + 15) / 16;
   dim3 grid((nblocks + kAwqBlocksPerCta - 1) / kAwqBlocksPerCta);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch ((M + 7) / 8) {
-    case 1: awq_gemv_kernel<1><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 2: awq_gemv_kernel<2><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 3: awq_gemv_kernel<3><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 4: awq_gemv_kernel<4><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 5: awq_gemv_kernel<5><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 6: awq_gemv_kernel<6><<<grid, kAwqThreads, 0, s>>>(p); break;
-    case 7: awq_gemv_kernel<7><<<grid, kAwqThreads, 0, s>>>(p); break;
-    default: awq_gemv_kernel<8><<<grid, kAwqThreads, 0, s>>>(p); break;
+  for (int m0 = 0; m0 < M; m0 += mc) {
+    const int mm = M - m0 < mc ? M - m0 : mc;
+    AwqParams p;
+    p.M = mm;
+    p.N = N;
+    p.K = K;
+    p.X = static_cast<const __nv_bfloat16*>(X) + static_cast<size_t>(m0) * K;
+    p.qweight = static_cast<const uint4*>(qweight);
+    p.sz = static_cast<const uint32_t*>(sz);
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.Y = static_cast<__nv_bfloat16*>(Y) + static_cast<size_t>(m0) * N;
+    p.status = d->status;
+    const size_t smem = awq_smem_bytes(mm, K);
+    if (mm <= 8)
+      awq_gemv_kernel<1><<<grid, kAwqThreads, smem, s>>>(p);
+    else
+      awq_gemv_kernel<2><<<grid, kAwqThreads, smem, s>>>(p);
   }
   return launch_status();
 }

@@ -6,14 +6,16 @@
 // the output).
 //
 // Persistent kernel: one CTA per SM walks 128 x 256 output tiles. Warp roles
-// (10 warps):
-//   warp 0     TMA producer: A/B code tiles [rows x 128 B] with 128-byte swizzle,
-//              A/B scale atoms by plain bulk copies, L2 chunks [32 x 256] bf16;
-//              runs ahead across tiles through a 3-stage ring
-//   warp 1     tensor-memory owner and MMA issuer (one thread)
-//   warps 2-5  low-rank staging: xl1 (float32) of the next tile as bf16 hi + lo
-//              operand tiles for the up-projection MMAs
-//   warps 6-9  epilogue: accumulator -> + bias -> bf16 / f32 -> global memory
+// (14 warps):
+//   warp 0      TMA producer: A/B code tiles [rows x 128 B] with 128-byte swizzle,
+//               A/B scale atoms by plain bulk copies, L2 chunks [16 x 256] bf16;
+//               runs ahead across tiles through a 3-stage ring
+//   warp 1      tensor-memory owner and MMA issuer (one thread)
+//   warps 2-5   low-rank staging: xl1 (float32) of the next tile as bf16 hi + lo
+//               operand tiles for the up-projection MMAs
+//   warps 6-13  epilogue, two warps per tensor-memory lane quadrant (one per
+//               128-column half): accumulator -> + bias -> bf16 / f32 -> swizzled
+//               shared-memory staging -> TMA store (coalesced, asynchronous)
 // Two 256-column accumulators share tensor memory with a 64-column overlap
 // ([0, 256) and [192, 448)); scale factors sit in [448, 496). The epilogue
 // drains the overlapped columns of a tile first and releases them, so the next
@@ -24,7 +26,9 @@
 
 namespace svdq {
 
-constexpr int kGmThreads = 320;
+constexpr int kGmThreads = 448;
+constexpr int kGmEpiWarps = 8;
+constexpr int kGmStageOut = 4096;                // epilogue staging bytes per warp
 constexpr int kGmBM = 128, kGmBN = 256;
 constexpr int kGmBKBytes = 128;  // 256 FP4 values per row per stage
 constexpr int kGmAStage = kGmBM * kGmBKBytes;   // 16 KB
@@ -33,9 +37,9 @@ constexpr int kGmSfaStage = 4 * 512;            // 4 atoms (one per 64-wide K bl
 constexpr int kGmSfbStage = 2 * 4 * 512;        // 2 row blocks x 4 atoms
 constexpr int kGmStageBytes = kGmAStage + kGmBStage + kGmSfaStage + kGmSfbStage;  // 54 KB
 constexpr int kGmStages = 3;
-constexpr int kGmLrK = 32;                                // low-rank K per chunk
-constexpr int kGmLrATile = kGmBM * kGmLrK * 2;            // 8 KB per bf16 tile
-constexpr int kGmLrBTile = kGmLrK * kGmBN * 2;            // 16 KB
+constexpr int kGmLrK = 16;                                // low-rank K per chunk
+constexpr int kGmLrATile = kGmBM * kGmLrK * 2;            // 4 KB per bf16 tile
+constexpr int kGmLrBTile = kGmLrK * kGmBN * 2;            // 8 KB
 // tensor-memory columns
 constexpr uint32_t kTmAcc1 = 192, kTmOverlap = 64, kTmSfa = 448, kTmSfb = 464, kTmCols = 512;
 
@@ -53,7 +57,7 @@ struct GemmParams {
 };
 
 struct GmSmem {
-  uint32_t ring, lr_a, lr_b, bars, tmem_slot, total;
+  uint32_t ring, lr_a, lr_b, out, bias, bars, tmem_slot, total;
 };
 
 __host__ __device__ constexpr GmSmem gm_smem_layout() {
@@ -61,7 +65,9 @@ __host__ __device__ constexpr GmSmem gm_smem_layout() {
   s.ring = 0;
   s.lr_b = kGmStages * kGmStageBytes;        // 1024-aligned (54 KB multiples)
   s.lr_a = s.lr_b + kGmLrBTile;
-  s.bars = s.lr_a + 2 * kGmLrATile;
+  s.out = s.lr_a + 2 * kGmLrATile;           // 1024-aligned
+  s.bias = s.out + kGmEpiWarps * kGmStageOut;  // 128 floats per epilogue warp
+  s.bars = s.bias + kGmEpiWarps * 128 * 4;
   s.tmem_slot = s.bars + 8 * (2 * kGmStages + 4);
   s.total = s.tmem_slot + 16;
   return s;
@@ -72,7 +78,8 @@ constexpr size_t kGmSmemBytes = gm_smem_layout().total + 1024;
 __global__ void __launch_bounds__(kGmThreads, 1)
     w4a4_nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                            const __grid_constant__ CUtensorMap tm_b,
-                           const __grid_constant__ CUtensorMap tm_l2, const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tm_l2,
+                           const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -116,10 +123,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     mbar_init(bar_lr_full, 1 + 4);  // producer (with tx) + 4 staging warps
     mbar_init(bar_lr_empty, 1);
     mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_free, 4);     // 4 epilogue warps
+    mbar_init(bar_acc_free, kGmEpiWarps);
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_y);
     if (p.r > 0) prefetch_tmap(&tm_l2);
   }
   if (warp == 1) {
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(bar_lr_full, kGmLrBTile);
           for (int nb = 0; nb < 4; ++nb)
-            tma_load_2d(lr_b + nb * 4096, &tm_l2, bar_lr_full, n0 + nb * 64, c * kGmLrK);
+            tma_load_2d(lr_b + nb * (kGmLrK * 128), &tm_l2, bar_lr_full, n0 + nb * 64, c * kGmLrK);
         }
         const int mb = m0 / 128;
         for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global) {
@@ -188,17 +196,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           ok = mbar_wait(bar_lr_full, lr_global & 1, p.status);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kGmLrK / 16; ++kk) {
-            // A (xl1 hi/lo): no-swizzle K-major, LBO 128 B (next 8 K), SBO 512 B (next 8 rows)
-            const uint64_t ah = smem_desc(lr_hi + kk * 256, 128, 512, kSwizzleNone);
-            const uint64_t al = smem_desc(lr_lo + kk * 256, 128, 512, kSwizzleNone);
-            // B (L2 chunk): MN-major, 128-byte swizzle; 64-wide N blocks 4096 B apart
-            // (LBO), 8-deep K groups 1024 B apart (SBO); 16 K = 2048 B.
-            const uint64_t bd = smem_desc(lr_b + kk * 2048, 4096, 1024, kSwizzle128B);
-            mma_f16(acc, ah, bd, id_lr, (c > 0 || kk > 0) ? 1u : 0u);
-            mma_f16(acc, al, bd, id_lr, 1u);
-          }
+          // A (xl1 hi/lo, 16 columns): no-swizzle K-major, the two 8-wide core
+          // matrices 128 B apart (LBO), 8-row groups 256 B apart (SBO).
+          // B (L2 chunk, 16 rows): MN-major, 128-byte swizzle; 64-wide N blocks
+          // 2048 B apart (LBO), the two 8-deep K groups 1024 B apart (SBO).
+          const uint64_t ah = smem_desc(lr_hi, 128, 256, kSwizzleNone);
+          const uint64_t al = smem_desc(lr_lo, 128, 256, kSwizzleNone);
+          const uint64_t bd = smem_desc(lr_b, kGmLrK * 128, 1024, kSwizzle128B);
+          mma_f16(acc, ah, bd, id_lr, c > 0 ? 1u : 0u);
+          mma_f16(acc, al, bd, id_lr, 1u);
           tc_commit(bar_lr_empty);
         }
         const uint32_t id_fp4 = idesc_nvfp4(128, n_tile);
@@ -244,9 +250,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                                                             c * kGmLrK);
 #pragma unroll
         for (int j = 0; j < kGmLrK / 4; ++j) {
-          // rows past M and columns past r (r % 32 == 16) contribute zeros
-          const float4 f = (m < p.M && c * kGmLrK + 4 * j < p.r) ? __ldg(src + j)
-                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 f = m < p.M ? __ldg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
           v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
         }
         ok = mbar_wait(bar_lr_empty, (lr_global & 1) ^ 1, p.status);
@@ -263,7 +267,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
             lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
           }
-          const uint32_t off = (trow >> 3) * 512 + cm * 128 + (trow & 7) * 16;
+          const uint32_t off = (trow >> 3) * 256 + cm * 128 + (trow & 7) * 16;
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lr_hi + off), "r"(hi[0]),
                        "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
                        : "memory");
@@ -278,68 +282,100 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;
-    const int trow = quad * 32 + lane;
+    // Each warp owns 4 of the tile's eight 32-column sub-tiles for its lane
+    // quadrant. The two sub-tiles shared with the other accumulator ([192, 256)
+    // of buffer 0, [0, 64) of buffer 1) come first, one in each half's warps, so
+    // the next tile's MMAs are let in after a single tensor-memory load per warp.
+    const int quad = warp & 3;          // tensor-memory lanes 32 quad .. 32 quad + 31
+    const int half = (warp - 6) >> 2;   // 0 or 1
+    const uint32_t out_buf = sbase + L.out + (warp - 6) * kGmStageOut;
+    float* bias_s = reinterpret_cast<float*>(smem + L.bias) + (warp - 6) * 128;  // [4][32]
     bool ok = true;
+    int stores = 0;
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
       const int n_tile = min(kGmBN, p.N - n0);
-      const int m = m0 + trow;
       const bool odd = i & 1;
       const uint32_t t_row = tmem + (odd ? kTmAcc1 : 0u) + (static_cast<uint32_t>(quad * 32) << 16);
+      // sub-tile order: the overlapped one, then three of the six others
+      int sub_col[4];
+      const int ovl = odd ? 0 : kGmBN - kTmOverlap;   // first overlapped column
+      sub_col[0] = ovl + 32 * half;
+      const int other0 = odd ? kTmOverlap : 0;        // first non-overlapped column
+      for (int t = 0; t < 3; ++t) sub_col[1 + t] = other0 + 32 * (3 * half + t);
+      // bias for this warp's sub-tiles, fetched before the accumulator is ready
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int n = n0 + sub_col[t] + lane;
+        bias_s[t * 32 + lane] = (p.bias != nullptr && n < p.N) ? __bfloat162float(p.bias[n]) : 0.0f;
+      }
+      __syncwarp();
       ok = mbar_wait(bar_acc_full, i & 1, p.status);
       if (!ok) break;
       tc_fence_after();
-      // columns of this tile, in 16-wide chunks, starting with the 64 columns
-      // shared with the other accumulator: [192, 256) of buffer 0, [0, 64) of buffer 1
-      const int first = odd ? 0 : kGmBN - kTmOverlap;
-      for (int step = 0; step < kGmBN / 16; ++step) {
-        const int j0 = (first + step * 16) % kGmBN;
-        uint32_t acc[16];
-        tmem_ld16(t_row + j0, acc);
+      for (int t = 0; t < 4; ++t) {
+        const int j0 = sub_col[t];
+        uint32_t acc[32];
+        tmem_ld32(t_row + j0, acc);
         tmem_ld_wait();
-        if (step == kTmOverlap / 16 - 1) {
-          // the overlapped columns are in registers: let the next tile's MMAs in
+        if (t == 0) {
+          // this warp's overlapped columns are in registers: let the next tile's MMAs in
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_acc_free);
         }
-        if (m >= p.M || j0 >= n_tile) continue;
-        float y[16];
-        const uint4* bsrc = reinterpret_cast<const uint4*>(p.bias + n0 + j0);
-        if (p.bias != nullptr) {
-          const uint4 b0 = __ldg(bsrc), b1 = __ldg(bsrc + 1);
-          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        if (j0 >= n_tile) continue;  // warp-uniform
+        float y[32];
+        const float4* bv = reinterpret_cast<const float4*>(bias_s + t * 32);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            y[2 * j] = __uint_as_float(acc[2 * j]) + __uint_as_float(bw[j] << 16);
-            y[2 * j + 1] = __uint_as_float(acc[2 * j + 1]) + __uint_as_float(bw[j] & 0xFFFF0000u);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(acc[j]);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 b = bv[q4];
+          y[4 * q4 + 0] = __uint_as_float(acc[4 * q4 + 0]) + b.x;
+          y[4 * q4 + 1] = __uint_as_float(acc[4 * q4 + 1]) + b.y;
+          y[4 * q4 + 2] = __uint_as_float(acc[4 * q4 + 2]) + b.z;
+          y[4 * q4 + 3] = __uint_as_float(acc[4 * q4 + 3]) + b.w;
         }
+        // stage the warp's 32 x 32 sub-tile in the TMA store's swizzled layout
+        uint32_t buf;
         if (p.out_f32) {
-          float* dst = reinterpret_cast<float*>(p.Y) + static_cast<size_t>(m) * p.ldy + n0 + j0;
+          buf = out_buf;  // one 4 KB buffer, rows of 128 B, 128-byte swizzle
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            reinterpret_cast<float4*>(dst)[j] =
-                make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+          for (int c = 0; c < 8; ++c)
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             buf + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                         "f"(y[4 * c]), "f"(y[4 * c + 1]), "f"(y[4 * c + 2]), "f"(y[4 * c + 3])
+                         : "memory");
         } else {
-          uint32_t pk[8];
+          buf = out_buf + (stores & 1) * 2048;  // two 2 KB buffers, rows of 64 B, 64-byte swizzle
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
             pk[j] = *reinterpret_cast<const uint32_t*>(&b);
           }
-          __nv_bfloat16* dst =
-              reinterpret_cast<__nv_bfloat16*>(p.Y) + static_cast<size_t>(m) * p.ldy + n0 + j0;
-          reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, buf, n0 + j0, m0 + quad * 32);
+          bulk_commit();
+        }
+        ++stores;
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

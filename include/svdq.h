@@ -143,7 +143,8 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
  *
  *   Y[m,n] = sum_k X[m,k] (q[n,k] - z[n,k/64]) s[n,k/64] + bias[n]
  *
- * X        device, bf16 [M, K] (row-major, K contiguous), 1 <= M <= 64
+ * X        device, bf16 [M, K] (row-major, K contiguous), 1 <= M <= 64; launches
+ *          cover up to 16 tokens each (fewer when K is large)
  * qweight  device, awq_qweight_bytes(N, K) bytes, fragment order from svdq_pack(AWQ)
  * sz       device, awq_sz_bytes(N, K) bytes, interleaved (s, z) from svdq_pack(AWQ)
  * bias     device, bf16 [N] or NULL
