@@ -53,7 +53,7 @@ __host__ __device__ constexpr size_t awq_stage_bytes() {
 }
 __host__ __device__ constexpr size_t awq_xrow_bytes(int K) { return static_cast<size_t>(K) * 2 + 16; }
 __host__ __device__ constexpr size_t awq_smem_bytes(int M, int K) {
-  return awq_stage_bytes() + static_cast<size_t>(M) * awq_xrow_bytes(K) +
+  return awq_stage_bytes() + static_cast<size_t>(M + 1) * awq_xrow_bytes(K) +
          static_cast<size_t>((M + 7) / 8) * 8 * (K / 64) * 4 + kAwqWarps * 8 + 128;
 }
 
@@ -81,19 +81,20 @@ __global__ void __launch_bounds__(kAwqThreads, 2) awq_gemv_kernel(const AwqParam
 
   uint8_t* wbuf = smem + static_cast<size_t>(warp) * kAwqBatch * kAwqGroupBytes;
   const size_t xrow_bytes = awq_xrow_bytes(p.K);
-  uint8_t* xsm = smem + awq_stage_bytes();                                    // [M][K + 8] bf16
-  float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M) * xrow_bytes);  // [kMB*8][G]
+  uint8_t* xsm = smem + awq_stage_bytes();  // [M + 1][K + 8] bf16, row M all zero
+  float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M + 1) * xrow_bytes);  // [kMB*8][G]
   const uint32_t bar = smem_u32(xs + kMB * 8 * G) + warp * 8;
 
   if (lane == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
   }
-  // stage X in shared memory
-  for (int t = threadIdx.x; t < p.M * (p.K / 8); t += kAwqThreads) {
+  // stage X in shared memory, plus one zero row that padding tokens read
+  for (int t = threadIdx.x; t < (p.M + 1) * (p.K / 8); t += kAwqThreads) {
     const int m = t / (p.K / 8), c = t % (p.K / 8);
     *reinterpret_cast<uint4*>(xsm + m * xrow_bytes + c * 16) =
-        __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.K) + c);
+        m < p.M ? __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.K) + c)
+                : make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();
   // per-group token sums xs[m][g] (rows >= M are zero)
@@ -122,14 +123,12 @@ __global__ void __launch_bounds__(kAwqThreads, 2) awq_gemv_kernel(const AwqParam
     for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
 
   if (blk < nblocks) {
-    // token rows this lane feeds as the B operand (rows >= M feed zeros)
-    uint32_t xrow[kMB];
-    bool xlive[kMB];
+    // token rows this lane feeds as the B operand (rows >= M read the zero row)
+    const uint32_t* xrow[kMB];
 #pragma unroll
     for (int b = 0; b < kMB; ++b) {
       const int m = b * 8 + r0;
-      xlive[b] = m < p.M;
-      xrow[b] = smem_u32(xsm) + static_cast<uint32_t>((xlive[b] ? m : 0) * xrow_bytes) + c0 * 2;
+      xrow[b] = reinterpret_cast<const uint32_t*>(xsm + (m < p.M ? m : p.M) * xrow_bytes) + c0 / 2;
     }
     uint32_t phase = 0;
     for (int g0 = g_begin; g0 < g_end; g0 += kAwqBatch) {
@@ -144,44 +143,41 @@ __global__ void __launch_bounds__(kAwqThreads, 2) awq_gemv_kernel(const AwqParam
       }
       if (!mbar_wait(bar, phase, p.status)) break;
       phase ^= 1;
-      const uint4* wq = reinterpret_cast<const uint4*>(wbuf);
-      const uint32_t* szs = reinterpret_cast<const uint32_t*>(wbuf + kAwqBatch * 512);
-      for (int j = 0; j < ng; ++j) {
-        const int g = g0 + j;
-        const uint4 w = wq[j * 32 + lane];
-        const uint32_t sz0 = szs[j * 16 + r0], sz8 = szs[j * 16 + r0 + 8];
-        const float s0 = __uint_as_float(sz0 << 16), s8 = __uint_as_float(sz8 << 16);
-        const float z0 = __uint_as_float(sz0 & 0xFFFF0000u) + 128.0f;
-        const float z8 = __uint_as_float(sz8 & 0xFFFF0000u) + 128.0f;
-        float part_acc[kMB][4];
+      const uint4* wq = reinterpret_cast<const uint4*>(wbuf) + lane;
+      const uint32_t* szs = reinterpret_cast<const uint32_t*>(wbuf + kAwqBatch * 512) + r0;
 #pragma unroll
-        for (int b = 0; b < kMB; ++b)
+      for (int j = 0; j < kAwqBatch; ++j) {
+        if (j < ng) {
+          const int g = g0 + j;
+          const uint4 w = wq[j * 32];
+          const uint32_t sz0 = szs[j * 16], sz8 = szs[j * 16 + 8];
+          float part_acc[kMB][4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) part_acc[b][e] = 0.0f;
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+          for (int b = 0; b < kMB; ++b)
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t a[4];
+            for (int e = 0; e < 4; ++e) part_acc[b][e] = 0.0f;
+          const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int pr = 0; pr < 4; ++pr)
-            a[pr] = ((words[ks] >> (4 * pr)) & 0x000F000Fu) | 0x43004300u;  // bf16 (128 + q) pairs
-          const int k = g * 64 + ks * 16;
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4];
+#pragma unroll
+            for (int pr = 0; pr < 4; ++pr)
+              a[pr] = ((words[ks] >> (4 * pr)) & 0x000F000Fu) | 0x43004300u;  // bf16 (128 + q) pairs
+            const int kw = (g * 64 + ks * 16) / 2;  // 32-bit word index of the fragment
+#pragma unroll
+            for (int b = 0; b < kMB; ++b) mma_bf16_16816(part_acc[b], a, xrow[b][kw], xrow[b][kw + 4]);
+          }
+          const float s0 = __uint_as_float(sz0 << 16), s8 = __uint_as_float(sz8 << 16);
+          const float z0 = __uint_as_float(sz0 & 0xFFFF0000u) + 128.0f;
+          const float z8 = __uint_as_float(sz8 & 0xFFFF0000u) + 128.0f;
 #pragma unroll
           for (int b = 0; b < kMB; ++b) {
-            uint32_t b0, b1;
-            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0) : "r"(xrow[b] + k * 2));
-            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1) : "r"(xrow[b] + k * 2 + 16));
-            if (!xlive[b]) b0 = b1 = 0u;
-            mma_bf16_16816(part_acc[b], a, b0, b1);
+            const float xs0 = xs[(b * 8 + c0) * G + g], xs1 = xs[(b * 8 + c0 + 1) * G + g];
+            acc[b][0] = fmaf(fmaf(-z0, xs0, part_acc[b][0]), s0, acc[b][0]);
+            acc[b][1] = fmaf(fmaf(-z0, xs1, part_acc[b][1]), s0, acc[b][1]);
+            acc[b][2] = fmaf(fmaf(-z8, xs0, part_acc[b][2]), s8, acc[b][2]);
+            acc[b][3] = fmaf(fmaf(-z8, xs1, part_acc[b][3]), s8, acc[b][3]);
           }
-        }
-#pragma unroll
-        for (int b = 0; b < kMB; ++b) {
-          const float xs0 = xs[(b * 8 + c0) * G + g], xs1 = xs[(b * 8 + c0 + 1) * G + g];
-          acc[b][0] = fmaf(fmaf(-z0, xs0, part_acc[b][0]), s0, acc[b][0]);
-          acc[b][1] = fmaf(fmaf(-z0, xs1, part_acc[b][1]), s0, acc[b][1]);
-          acc[b][2] = fmaf(fmaf(-z8, xs0, part_acc[b][2]), s8, acc[b][2]);
-          acc[b][3] = fmaf(fmaf(-z8, xs1, part_acc[b][3]), s8, acc[b][3]);
         }
       }
       __syncwarp();  // every lane is done with the staging buffer before it is refilled

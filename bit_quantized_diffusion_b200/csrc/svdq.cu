@@ -186,25 +186,27 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   auto fits = [&](int st, int budget) {
     return st >= 2 && fixed + st * stage_bytes <= budget && red_bytes <= st * stage_bytes;
   };
-  int stages = 0, per_sm = 1;
+  // Two configurations: two CTAs per SM (ring in half the shared memory, at
+  // least 3 stages) or one CTA per SM (up to 8 stages). Two per SM is used only
+  // when the grid has more CTAs than SMs: the block scheduler fills SMs two at a
+  // time, so a smaller grid would leave SMs idle.
+  int stages2 = 0, stages1 = 0;
   const int half_budget = 113 * 1024, full_budget = 227 * 1024;
-  for (int st = 8; st >= 3; --st)
-    if (fits(st, half_budget)) { stages = st; per_sm = 2; break; }
-  if (stages == 0)
-    for (int st = 8; st >= 2; --st)
-      if (fits(st, full_budget)) { stages = st; break; }
-  if (stages == 0) return SVDQ_ERR_UNSUPPORTED;
+  for (int st = 8; st >= 3 && stages2 == 0; --st)
+    if (fits(st, half_budget)) stages2 = st;
+  for (int st = 8; st >= 2 && stages1 == 0; --st)
+    if (fits(st, full_budget)) stages1 = st;
+  if (stages1 == 0) return SVDQ_ERR_UNSUPPORTED;
+  // K split: the largest power of two (<= 8, <= K/64) whose CTAs fit in one wave
+  const int max_ctas = (stages2 ? 2 : 1) * d->num_sms;
+  int ksplit = 1;
+  while (ksplit * 2 <= 8 && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= max_ctas)
+    ksplit *= 2;
+  const bool two_per_sm = stages2 != 0 && row_blocks * ksplit > d->num_sms;
+  const int stages = two_per_sm ? stages2 : stages1;
+  const int per_sm = two_per_sm ? 2 : 1;
   const size_t smem_bytes = qa_smem_bytes(r, stages);
   auto kern = format == SVDQ_NVFP4_G16 ? quantize_act_kernel<0> : quantize_act_kernel<1>;
-
-  // K split: the largest power of two (<= 8, <= 4 with two CTAs per SM so a
-  // cluster's CTAs fit in one GPC alongside others, <= K/64) whose CTAs fit in
-  // one wave of the SMs.
-  const int slots = per_sm * d->num_sms;
-  const int s_cap = per_sm == 2 ? 4 : 8;
-  int ksplit = 1;
-  while (ksplit * 2 <= s_cap && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= slots)
-    ksplit *= 2;
   if (std::getenv("SVDQ_DEBUG") != nullptr)
     std::fprintf(stderr, "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d\n",
                  M, K, r, stages, per_sm, ksplit, ksplit * row_blocks);

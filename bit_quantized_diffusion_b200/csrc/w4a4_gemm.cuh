@@ -8,11 +8,15 @@
 // Persistent kernel: one CTA per SM walks 128 x 256 output tiles. Warp roles
 // (14 warps):
 //   warp 0      TMA producer: A/B code tiles [rows x 128 B] with 128-byte swizzle,
-//               A/B scale atoms by plain bulk copies, L2 chunks [16 x 256] bf16;
+//               A/B scale atoms by plain bulk copies, L2 chunks [32 x 256] bf16;
 //               runs ahead across tiles through a 3-stage ring
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
-//   warps 2-5   low-rank staging: xl1 (float32) of the next tile as bf16 hi + lo
-//               operand tiles for the up-projection MMAs
+//   warps 2-5   low-rank staging: xl1 (float32) as bf16 hi + lo operand tiles
+//               for the up-projection MMAs
+// Each tile is a sequence of ring slots: K/256 FP4 slots, then ceil(r/32)
+// low-rank slots holding an L2 chunk (by TMA) and the matching xl1 hi/lo tiles
+// (by the staging warps). Every slot's "full" barrier counts the producer and
+// the four staging warps, so both kinds of slot flow through one pipeline.
 //   warps 6-13  epilogue, two warps per tensor-memory lane quadrant (one per
 //               128-column half): accumulator -> + bias -> bf16 / f32 -> swizzled
 //               shared-memory staging -> TMA store (coalesced, asynchronous)
@@ -37,9 +41,9 @@ constexpr int kGmSfaStage = 4 * 512;            // 4 atoms (one per 64-wide K bl
 constexpr int kGmSfbStage = 2 * 4 * 512;        // 2 row blocks x 4 atoms
 constexpr int kGmStageBytes = kGmAStage + kGmBStage + kGmSfaStage + kGmSfbStage;  // 54 KB
 constexpr int kGmStages = 3;
-constexpr int kGmLrK = 16;                                // low-rank K per chunk
-constexpr int kGmLrATile = kGmBM * kGmLrK * 2;            // 4 KB per bf16 tile
-constexpr int kGmLrBTile = kGmLrK * kGmBN * 2;            // 8 KB
+constexpr int kGmLrK = 32;                                // low-rank K per ring slot
+constexpr int kGmLrBTile = kGmLrK * kGmBN * 2;            // 16 KB, slot offset 0
+constexpr int kGmLrATile = kGmBM * kGmLrK * 2;            // 8 KB per bf16 tile (hi, lo)
 // tensor-memory columns
 constexpr uint32_t kTmAcc1 = 192, kTmOverlap = 64, kTmSfa = 448, kTmSfb = 464, kTmCols = 512;
 
@@ -57,18 +61,16 @@ struct GemmParams {
 };
 
 struct GmSmem {
-  uint32_t ring, lr_a, lr_b, out, bias, bars, tmem_slot, total;
+  uint32_t ring, out, bias, bars, tmem_slot, total;
 };
 
 __host__ __device__ constexpr GmSmem gm_smem_layout() {
   GmSmem s{};
   s.ring = 0;
-  s.lr_b = kGmStages * kGmStageBytes;        // 1024-aligned (54 KB multiples)
-  s.lr_a = s.lr_b + kGmLrBTile;
-  s.out = s.lr_a + 2 * kGmLrATile;           // 1024-aligned
+  s.out = kGmStages * kGmStageBytes;         // 1024-aligned (54 KB multiples)
   s.bias = s.out + kGmEpiWarps * kGmStageOut;  // 128 floats per epilogue warp
   s.bars = s.bias + kGmEpiWarps * 128 * 4;
-  s.tmem_slot = s.bars + 8 * (2 * kGmStages + 4);
+  s.tmem_slot = s.bars + 8 * (2 * kGmStages + 2);
   s.total = s.tmem_slot + 16;
   return s;
 }
@@ -107,21 +109,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   auto sfb_st = [&](int s) { return sfa_st(s) + kGmSfaStage; };
   auto bar_full = [&](int s) { return sbase + L.bars + 8 * s; };
   auto bar_empty = [&](int s) { return sbase + L.bars + 8 * (kGmStages + s); };
-  const uint32_t bar_lr_full = sbase + L.bars + 8 * (2 * kGmStages);
-  const uint32_t bar_lr_empty = bar_lr_full + 8;
-  const uint32_t bar_acc_full = bar_lr_full + 16;
-  const uint32_t bar_acc_free = bar_lr_full + 24;
-  const uint32_t lr_b = sbase + L.lr_b;
-  const uint32_t lr_hi = sbase + L.lr_a, lr_lo = lr_hi + kGmLrATile;
+  const uint32_t bar_acc_full = sbase + L.bars + 8 * (2 * kGmStages);
+  const uint32_t bar_acc_free = bar_acc_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGmStages; ++s) {
-      mbar_init(bar_full(s), 1);
+      mbar_init(bar_full(s), 1 + 4);  // producer (with tx) + 4 staging warps
       mbar_init(bar_empty(s), 1);
     }
-    mbar_init(bar_lr_full, 1 + 4);  // producer (with tx) + 4 staging warps
-    mbar_init(bar_lr_empty, 1);
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_free, kGmEpiWarps);
     fence_barrier_init();
@@ -143,34 +139,37 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     // ------------------------------------------------------------ producer
     if (elect_one()) {
       bool ok = true;
-      int kt_global = 0, lr_global = 0;
+      int kt_global = 0;
       for (int i = 0; i < my_tiles && ok; ++i) {
         int m0, n0;
         tile_mn(i, m0, n0);
         const int n_tile = min(kGmBN, p.N - n0);
         const int n_sfb = n_tile > 128 ? 2 : 1;
-        for (int c = 0; c < lr_chunks && ok; ++c, ++lr_global) {
-          ok = mbar_wait(bar_lr_empty, (lr_global & 1) ^ 1, p.status);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar_lr_full, kGmLrBTile);
-          for (int nb = 0; nb < 4; ++nb)
-            tma_load_2d(lr_b + nb * (kGmLrK * 128), &tm_l2, bar_lr_full, n0 + nb * 64, c * kGmLrK);
-        }
         const int mb = m0 / 128;
-        for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global) {
+        for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
           const int s = kt_global % kGmStages;
           ok = mbar_wait(bar_empty(s), ((kt_global / kGmStages) & 1) ^ 1, p.status);
           if (!ok) break;
-          const int nkb = min(4, kblocks - 4 * kt);
-          mbar_arrive_expect_tx(bar_full(s), kGmAStage + kGmBStage + nkb * 512 * (1 + n_sfb));
-          tma_load_2d(a_st(s), &tm_a, bar_full(s), kt * kGmBKBytes, m0);
-          tma_load_2d(b_st(s), &tm_b, bar_full(s), kt * kGmBKBytes, n0);
-          bulk_load(sfa_st(s), p.a_scales + (static_cast<size_t>(mb) * kblocks + 4 * kt) * 512,
-                    nkb * 512, bar_full(s));
-          for (int j = 0; j < n_sfb; ++j)
-            bulk_load(sfb_st(s) + j * 2048,
-                      p.w_scales + (static_cast<size_t>(n0 / 128 + j) * kblocks + 4 * kt) * 512,
+          if (kt < ktiles) {
+            const int nkb = min(4, kblocks - 4 * kt);
+            mbar_arrive_expect_tx(bar_full(s), kGmAStage + kGmBStage + nkb * 512 * (1 + n_sfb));
+            tma_load_2d(a_st(s), &tm_a, bar_full(s), kt * kGmBKBytes, m0);
+            tma_load_2d(b_st(s), &tm_b, bar_full(s), kt * kGmBKBytes, n0);
+            bulk_load(sfa_st(s), p.a_scales + (static_cast<size_t>(mb) * kblocks + 4 * kt) * 512,
                       nkb * 512, bar_full(s));
+            for (int j = 0; j < n_sfb; ++j)
+              bulk_load(sfb_st(s) + j * 2048,
+                        p.w_scales + (static_cast<size_t>(n0 / 128 + j) * kblocks + 4 * kt) * 512,
+                        nkb * 512, bar_full(s));
+          } else {
+            // low-rank slot: L2 rows [32 c, 32 c + 32) x columns [n0, n0 + 256),
+            // four 64-wide boxes (rows past r read as zero)
+            const int c = kt - ktiles;
+            mbar_arrive_expect_tx(bar_full(s), kGmLrBTile);
+            for (int nb = 0; nb < 4; ++nb)
+              tma_load_2d(stage(s) + nb * (kGmLrK * 128), &tm_l2, bar_full(s), n0 + nb * 64,
+                          c * kGmLrK);
+          }
         }
       }
     }
@@ -179,7 +178,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     if (elect_one()) {
       bool ok = true;
       const uint32_t id_lr = idesc_bf16_f32(128, kGmBN, false, true);
-      int kt_global = 0, lr_global = 0;
+      int kt_global = 0;
       for (int i = 0; i < my_tiles && ok; ++i) {
         int m0, n0;
         tile_mn(i, m0, n0);
@@ -192,41 +191,40 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           if (!ok) break;
         }
         tc_fence_after();
-        for (int c = 0; c < lr_chunks && ok; ++c, ++lr_global) {
-          ok = mbar_wait(bar_lr_full, lr_global & 1, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          // A (xl1 hi/lo, 16 columns): no-swizzle K-major, the two 8-wide core
-          // matrices 128 B apart (LBO), 8-row groups 256 B apart (SBO).
-          // B (L2 chunk, 16 rows): MN-major, 128-byte swizzle; 64-wide N blocks
-          // 2048 B apart (LBO), the two 8-deep K groups 1024 B apart (SBO).
-          const uint64_t ah = smem_desc(lr_hi, 128, 256, kSwizzleNone);
-          const uint64_t al = smem_desc(lr_lo, 128, 256, kSwizzleNone);
-          const uint64_t bd = smem_desc(lr_b, kGmLrK * 128, 1024, kSwizzle128B);
-          mma_f16(acc, ah, bd, id_lr, c > 0 ? 1u : 0u);
-          mma_f16(acc, al, bd, id_lr, 1u);
-          tc_commit(bar_lr_empty);
-        }
         const uint32_t id_fp4 = idesc_nvfp4(128, n_tile);
-        for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global) {
+        for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
           const int s = kt_global % kGmStages;
           ok = mbar_wait(bar_full(s), (kt_global / kGmStages) & 1, p.status);
           if (!ok) break;
           tc_fence_after();
-          const int nkb = min(4, kblocks - 4 * kt);
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_cp_32x128b_warpx4(tmem + kTmSfa + 4 * kb,
-                                 smem_desc(sfa_st(s) + kb * 512, 128, 128, kSwizzleNone));
-            for (int j = 0; j < n_sfb; ++j)
-              tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb + 4 * j,
-                                   smem_desc(sfb_st(s) + j * 2048 + kb * 512, 128, 128,
-                                             kSwizzleNone));
-          }
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint64_t ad = smem_desc(a_st(s) + kb * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(b_st(s) + kb * 32, 16, 1024, kSwizzle128B);
-            mma_nvfp4(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
-                      (lr_chunks > 0 || kt > 0 || kb > 0) ? 1u : 0u);
+          if (kt < ktiles) {
+            const int nkb = min(4, kblocks - 4 * kt);
+            for (int kb = 0; kb < nkb; ++kb) {
+              tc_cp_32x128b_warpx4(tmem + kTmSfa + 4 * kb,
+                                   smem_desc(sfa_st(s) + kb * 512, 128, 128, kSwizzleNone));
+              for (int j = 0; j < n_sfb; ++j)
+                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb + 4 * j,
+                                     smem_desc(sfb_st(s) + j * 2048 + kb * 512, 128, 128,
+                                               kSwizzleNone));
+            }
+            for (int kb = 0; kb < nkb; ++kb) {
+              const uint64_t ad = smem_desc(a_st(s) + kb * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(b_st(s) + kb * 32, 16, 1024, kSwizzle128B);
+              mma_nvfp4(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
+                        (kt > 0 || kb > 0) ? 1u : 0u);
+            }
+          } else {
+            // low-rank slot: B = L2 chunk (MN-major, 128-byte swizzle; 64-wide N
+            // blocks 4096 B apart = LBO, 8-deep K groups 1024 B apart = SBO);
+            // A = xl1 hi / lo (no-swizzle K-major: K-adjacent core matrices 128 B
+            // apart = LBO, 8-row groups 512 B apart = SBO)
+            const uint32_t a_hi = stage(s) + kGmLrBTile, a_lo = a_hi + kGmLrATile;
+#pragma unroll
+            for (int kk = 0; kk < kGmLrK / 16; ++kk) {
+              const uint64_t bd = smem_desc(stage(s) + kk * 2048, kGmLrK * 128, 1024, kSwizzle128B);
+              mma_f16(acc, smem_desc(a_hi + kk * 256, 128, 512, kSwizzleNone), bd, id_lr, 1u);
+              mma_f16(acc, smem_desc(a_lo + kk * 256, 128, 512, kSwizzleNone), bd, id_lr, 1u);
+            }
           }
           tc_commit(bar_empty(s));
         }
@@ -238,46 +236,55 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int quad = warp & 3;
     const int trow = quad * 32 + lane;
     bool ok = true;
-    int lr_global = 0;
+    int kt_global = 0;
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
       const int m = m0 + trow;
-      for (int c = 0; c < lr_chunks && ok; ++c, ++lr_global) {
-        // load before waiting: the global read overlaps the wait for the buffer
+      for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
+        const int s = kt_global % kGmStages;
         float v[kGmLrK];
-        const float4* src = reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r +
-                                                            c * kGmLrK);
+        const int c = kt - ktiles;
+        if (c >= 0) {
+          // load before waiting: the global read overlaps the wait for the slot
+          const float4* src = reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r +
+                                                              c * kGmLrK);
 #pragma unroll
-        for (int j = 0; j < kGmLrK / 4; ++j) {
-          const float4 f = m < p.M ? __ldg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
-        }
-        ok = mbar_wait(bar_lr_empty, (lr_global & 1) ^ 1, p.status);
-        if (!ok) break;
-#pragma unroll
-        for (int cm = 0; cm < kGmLrK / 8; ++cm) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float x0 = v[8 * cm + 2 * j], x1 = v[8 * cm + 2 * j + 1];
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(hb);
-            const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-            hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
-            lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
+          for (int j = 0; j < kGmLrK / 4; ++j) {
+            // rows past M and columns past r (r % 32 == 16) contribute zeros
+            const float4 f = (m < p.M && c * kGmLrK + 4 * j < p.r) ? __ldg(src + j)
+                                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
           }
-          const uint32_t off = (trow >> 3) * 256 + cm * 128 + (trow & 7) * 16;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lr_hi + off), "r"(hi[0]),
-                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
-                       : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lr_lo + off), "r"(lo[0]),
-                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
-                       : "memory");
         }
-        fence_proxy_async_smem();
+        ok = mbar_wait(bar_empty(s), ((kt_global / kGmStages) & 1) ^ 1, p.status);
+        if (!ok) break;
+        if (c >= 0) {
+          const uint32_t a_hi = stage(s) + kGmLrBTile, a_lo = a_hi + kGmLrATile;
+#pragma unroll
+          for (int cm = 0; cm < kGmLrK / 8; ++cm) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float x0 = v[8 * cm + 2 * j], x1 = v[8 * cm + 2 * j + 1];
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+              const float2 hf = __bfloat1622float2(hb);
+              const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+              hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
+              lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
+            }
+            const uint32_t off = (trow >> 3) * 512 + cm * 128 + (trow & 7) * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi + off), "r"(hi[0]),
+                         "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
+                         : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo + off), "r"(lo[0]),
+                         "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_lr_full);
+        if (lane == 0) mbar_arrive(bar_full(s));
       }
     }
   } else {
