@@ -27,6 +27,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  int gemm_pairs = 0;  // co-resident clusters of the CTA-pair GEMM
   uint32_t* status = nullptr;
 };
 
@@ -65,14 +66,44 @@ svdq_status device_setup(DeviceInfo** out) {
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(quantize_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kGmSmemBytes)) != cudaSuccess)
+        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(GmCfg<false>::kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(GmCfg<true>::kSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     if (cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(awq_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess)
       return SVDQ_ERR_CUDA;
+    {
+      // how many 2-CTA clusters of the pair GEMM can be resident at once (a
+      // persistent grid larger than that would run its last clusters late)
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (d.num_sms / 2), 1, 1);
+      q.blockDim = dim3(kGmThreads, 1, 1);
+      q.dynamicSmemBytes = GmCfg<true>::kSmemBytes;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 2;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, w4a4_nvfp4_gemm_kernel<true>, &q) !=
+              cudaSuccess ||
+          clusters <= 0) {
+        (void)cudaGetLastError();
+        clusters = d.num_sms / 2;
+      }
+      d.gemm_pairs = clusters < d.num_sms / 2 ? clusters : d.num_sms / 2;
+      if (std::getenv("SVDQ_DEBUG") != nullptr)
+        std::fprintf(stderr, "svdq: %d SMs, %d co-resident GEMM CTA pairs\n", d.num_sms,
+                     d.gemm_pairs);
+    }
     d.status = static_cast<uint32_t*>(st);
     d.ready = true;
   }
@@ -263,11 +294,21 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
 
-  CUtensorMap tm_a, tm_b, tm_l2, tm_y;
+  // pairs of CTAs (cta_group::2, 256-row tiles) unless M fits one CTA's 128 rows
+  const bool pair = M > kGmBM;
+  const int ctas = pair ? 2 : 1;
+  const int b_rows = kGmBN / ctas;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y;
+  const uint64_t kb = static_cast<uint64_t>(K / 64);
   if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, kGmBKBytes,
                     kGmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, kGmBKBytes,
-                    kGmBN, CU_TENSOR_MAP_SWIZZLE_128B))
+                    b_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      // scale atoms as rows of 256 B (two rows per 512-byte atom), 8 rows = 4 atoms per box
+      !make_tmap_2d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 256, pad128(M) / 128 * kb * 2,
+                    256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 256, pad128(N) / 128 * kb * 2,
+                    256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, N, r,
@@ -287,19 +328,35 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.N = N;
   p.K = K;
   p.r = r;
-  p.a_scales = static_cast<const uint8_t*>(a_scales);
-  p.w_scales = static_cast<const uint8_t*>(w_scales);
   p.xl1 = xl1;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
-  p.Y = Y;
-  p.ldy = ldy;
-  p.out_f32 = out == SVDQ_OUT_F32;
+  p.out_f32 = f32;
   p.status = d->status;
-  p.tiles_m = (M + kGmBM - 1) / kGmBM;
+  p.tiles_m = (M + kGmBM * ctas - 1) / (kGmBM * ctas);
   p.tiles = p.tiles_m * ((N + kGmBN - 1) / kGmBN);
-  const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
-  w4a4_nvfp4_gemm_kernel<<<grid, kGmThreads, kGmSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      tm_a, tm_b, tm_l2, tm_y, p);
+  const int max_units = pair ? d->gemm_pairs : d->num_sms;
+  const int units = p.tiles < max_units ? p.tiles : max_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units * ctas, 1, 1);
+  cfg.blockDim = dim3(kGmThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair ? GmCfg<true>::kSmemBytes : GmCfg<false>::kSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pair ? 1 : 0;
+  const cudaError_t e =
+      pair ? cudaLaunchKernelEx(&cfg, w4a4_nvfp4_gemm_kernel<true>, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2,
+                                tm_y, p)
+           : cudaLaunchKernelEx(&cfg, w4a4_nvfp4_gemm_kernel<false>, tm_a, tm_b, tm_sfa, tm_sfb,
+                                tm_l2, tm_y, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
   return launch_status();
 }
 

@@ -5,21 +5,27 @@
 // (Nunchaku README, "Engine design" (b): up projection and 4-bit compute share
 // the output).
 //
-// Persistent kernel: one CTA per SM walks 128 x 256 output tiles. Warp roles
-// (14 warps):
+// Persistent kernel. In pair mode (kPair) a cluster of two CTAs on two SMs
+// computes 256 x 256 output tiles with cta_group::2 MMAs: each CTA stages its
+// own 128 rows of A and its own 128 of the tile's 256 B rows, the pair's tensor
+// cores exchange the B halves, and each CTA's tensor memory accumulates its 128
+// rows. Per CTA that halves the B traffic and the B shared memory of a stage,
+// which buys a 4-stage ring. Without kPair one CTA computes 128 x 256 tiles.
+//
+// Warp roles per CTA (14 warps):
 //   warp 0      TMA producer: A/B code tiles [rows x 128 B] with 128-byte swizzle,
-//               A/B scale atoms by plain bulk copies, L2 chunks [32 x 256] bf16;
-//               runs ahead across tiles through a 3-stage ring
-//   warp 1      tensor-memory owner and MMA issuer (one thread)
+//               A/B scale atoms, L2 chunks [32 x 128 or 256] bf16; runs ahead
+//               across tiles through the ring
+//   warp 1      tensor-memory owner; in the leader CTA also the MMA issuer (one
+//               thread)
 //   warps 2-5   low-rank staging: xl1 (float32) as bf16 hi + lo operand tiles
-//               for the up-projection MMAs
+//   warps 6-13  epilogue, two warps per tensor-memory lane quadrant: accumulator
+//               -> + bias -> bf16 / f32 -> swizzled shared memory -> TMA store
 // Each tile is a sequence of ring slots: K/256 FP4 slots, then ceil(r/32)
 // low-rank slots holding an L2 chunk (by TMA) and the matching xl1 hi/lo tiles
-// (by the staging warps). Every slot's "full" barrier counts the producer and
-// the four staging warps, so both kinds of slot flow through one pipeline.
-//   warps 6-13  epilogue, two warps per tensor-memory lane quadrant (one per
-//               128-column half): accumulator -> + bias -> bf16 / f32 -> swizzled
-//               shared-memory staging -> TMA store (coalesced, asynchronous)
+// (by the staging warps). A slot's "full" barrier (the leader's) counts the
+// leader's producer, whose expected bytes cover both CTAs' loads, and every
+// staging warp of the pair; the MMA commit frees the slot in both CTAs.
 // Two 256-column accumulators share tensor memory with a 64-column overlap
 // ([0, 256) and [192, 448)); scale factors sit in [448, 496). The epilogue
 // drains the overlapped columns of a tile first and releases them, so the next
@@ -33,105 +39,113 @@ namespace svdq {
 constexpr int kGmThreads = 448;
 constexpr int kGmEpiWarps = 8;
 constexpr int kGmStageOut = 4096;                // epilogue staging bytes per warp
-constexpr int kGmBM = 128, kGmBN = 256;
-constexpr int kGmBKBytes = 128;  // 256 FP4 values per row per stage
-constexpr int kGmAStage = kGmBM * kGmBKBytes;   // 16 KB
-constexpr int kGmBStage = kGmBN * kGmBKBytes;   // 32 KB
-constexpr int kGmSfaStage = 4 * 512;            // 4 atoms (one per 64-wide K block)
-constexpr int kGmSfbStage = 2 * 4 * 512;        // 2 row blocks x 4 atoms
-constexpr int kGmStageBytes = kGmAStage + kGmBStage + kGmSfaStage + kGmSfbStage;  // 54 KB
-constexpr int kGmStages = 3;
-constexpr int kGmLrK = 32;                                // low-rank K per ring slot
-constexpr int kGmLrBTile = kGmLrK * kGmBN * 2;            // 16 KB, slot offset 0
-constexpr int kGmLrATile = kGmBM * kGmLrK * 2;            // 8 KB per bf16 tile (hi, lo)
+constexpr int kGmBM = 128, kGmBN = 256;          // rows per CTA, columns per tile
+constexpr int kGmBKBytes = 128;                  // 256 FP4 values per row per stage
+constexpr int kGmAStage = kGmBM * kGmBKBytes;    // 16 KB
+constexpr int kGmSfaStage = 4 * 512;             // 4 atoms (one per 64-wide K block)
+constexpr int kGmSfbStage = 2 * 4 * 512;         // 2 row blocks x 4 atoms
+constexpr int kGmLrK = 32;                       // low-rank K per ring slot
+constexpr int kGmLrATile = kGmBM * kGmLrK * 2;   // 8 KB per bf16 tile (hi, lo)
 // tensor-memory columns
 constexpr uint32_t kTmAcc1 = 192, kTmOverlap = 64, kTmSfa = 448, kTmSfb = 464, kTmCols = 512;
 
+template <bool kPair>
+struct GmCfg {
+  static constexpr int kCtas = kPair ? 2 : 1;
+  static constexpr int kBRows = kGmBN / kCtas;                // B rows staged per CTA
+  static constexpr int kBStage = kBRows * kGmBKBytes;
+  static constexpr int kStageBytes = kGmAStage + kBStage + kGmSfaStage + kGmSfbStage;
+  static constexpr int kStages = kPair ? 4 : 3;
+  static constexpr int kLrBTile = kGmLrK * kBRows * 2;        // L2 chunk, slot offset 0
+  static constexpr uint32_t kOut = kStages * kStageBytes;     // 1024-aligned
+  static constexpr uint32_t kBias = kOut + kGmEpiWarps * kGmStageOut;
+  static constexpr uint32_t kBars = kBias + kGmEpiWarps * 128 * 4;
+  static constexpr uint32_t kTmemSlot = kBars + 8 * (2 * kStages + 2);
+  static constexpr size_t kSmemBytes = kTmemSlot + 16 + 1024;
+  static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+  static_assert(kLrBTile + 2 * kGmLrATile <= kStageBytes, "a low-rank slot fits in a stage");
+};
+
 struct GemmParams {
   int M, N, K, r;
-  int tiles_m, tiles;
-  const uint8_t* a_scales;
-  const uint8_t* w_scales;
+  int tiles_m, tiles;      // tiles of kCtas * 128 rows x 256 columns
   const float* xl1;
   const __nv_bfloat16* bias;
-  void* Y;
-  int ldy;
   int out_f32;
   uint32_t* status;
 };
 
-struct GmSmem {
-  uint32_t ring, out, bias, bars, tmem_slot, total;
-};
-
-__host__ __device__ constexpr GmSmem gm_smem_layout() {
-  GmSmem s{};
-  s.ring = 0;
-  s.out = kGmStages * kGmStageBytes;         // 1024-aligned (54 KB multiples)
-  s.bias = s.out + kGmEpiWarps * kGmStageOut;  // 128 floats per epilogue warp
-  s.bars = s.bias + kGmEpiWarps * 128 * 4;
-  s.tmem_slot = s.bars + 8 * (2 * kGmStages + 2);
-  s.total = s.tmem_slot + 16;
-  return s;
-}
-
-constexpr size_t kGmSmemBytes = gm_smem_layout().total + 1024;
-
+template <bool kPair>
 __global__ void __launch_bounds__(kGmThreads, 1)
     w4a4_nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                            const __grid_constant__ CUtensorMap tm_b,
+                           const __grid_constant__ CUtensorMap tm_sfa,
+                           const __grid_constant__ CUtensorMap tm_sfb,
                            const __grid_constant__ CUtensorMap tm_l2,
                            const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+  using Cfg = GmCfg<kPair>;
+  constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  constexpr GmSmem L = gm_smem_layout();
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   const int kblocks = p.K / 64;                      // 64-wide scale atoms along K
   const int ktiles = (kblocks + 3) / 4;
-  const int lr_chunks = p.r / kGmLrK + ((p.r % kGmLrK) ? 1 : 0);
-  // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...; M fastest
-  const int my_tiles = p.tiles > static_cast<int>(blockIdx.x)
-                           ? (p.tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
-                           : 0;
+  const int lr_chunks = (p.r + kGmLrK - 1) / kGmLrK;
+  const int slots = ktiles + lr_chunks;              // ring slots per tile
+  const int unit = blockIdx.x / Cfg::kCtas;          // this CTA (pair)'s scheduling unit
+  const int units = gridDim.x / Cfg::kCtas;
+  // this unit's tiles: unit, unit + units, ...; M fastest
+  const int my_tiles = p.tiles > unit ? (p.tiles - 1 - unit) / units + 1 : 0;
   auto tile_mn = [&](int i, int& m0, int& n0) {
-    const int t = blockIdx.x + i * gridDim.x;
-    m0 = (t % p.tiles_m) * kGmBM;
+    const int t = unit + i * units;
+    m0 = (t % p.tiles_m) * (kGmBM * Cfg::kCtas);
     n0 = (t / p.tiles_m) * kGmBN;
   };
 
-  auto stage = [&](int s) { return sbase + L.ring + s * kGmStageBytes; };
+  auto stage = [&](int s) { return sbase + s * Cfg::kStageBytes; };
   auto a_st = [&](int s) { return stage(s); };
   auto b_st = [&](int s) { return stage(s) + kGmAStage; };
-  auto sfa_st = [&](int s) { return stage(s) + kGmAStage + kGmBStage; };
+  auto sfa_st = [&](int s) { return stage(s) + kGmAStage + Cfg::kBStage; };
   auto sfb_st = [&](int s) { return sfa_st(s) + kGmSfaStage; };
-  auto bar_full = [&](int s) { return sbase + L.bars + 8 * s; };
-  auto bar_empty = [&](int s) { return sbase + L.bars + 8 * (kGmStages + s); };
-  const uint32_t bar_acc_full = sbase + L.bars + 8 * (2 * kGmStages);
+  auto bar_full = [&](int s) { return sbase + Cfg::kBars + 8 * s; };
+  auto bar_empty = [&](int s) { return sbase + Cfg::kBars + 8 * (NS + s); };
+  const uint32_t bar_acc_full = sbase + Cfg::kBars + 8 * (2 * NS);
   const uint32_t bar_acc_free = bar_acc_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
+  // the leader's copies of the pipeline barriers, as seen from this CTA
+  auto lead = [&](uint32_t a) { return kPair ? map_peer_smem(a, 0) : a; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kTmemSlot);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGmStages; ++s) {
-      mbar_init(bar_full(s), 1 + 4);  // producer (with tx) + 4 staging warps
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full(s), 1 + 4 * Cfg::kCtas);  // leader producer (with tx) + staging warps
       mbar_init(bar_empty(s), 1);
     }
     mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_free, kGmEpiWarps);
+    mbar_init(bar_acc_free, kGmEpiWarps * Cfg::kCtas);
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb);
     prefetch_tmap(&tm_y);
     if (p.r > 0) prefetch_tmap(&tm_l2);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), kTmCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), kTmCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync(); else __syncthreads();  // barriers initialised in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -143,92 +157,111 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       for (int i = 0; i < my_tiles && ok; ++i) {
         int m0, n0;
         tile_mn(i, m0, n0);
-        const int n_tile = min(kGmBN, p.N - n0);
-        const int n_sfb = n_tile > 128 ? 2 : 1;
-        const int mb = m0 / 128;
-        for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
-          const int s = kt_global % kGmStages;
-          ok = mbar_wait(bar_empty(s), ((kt_global / kGmStages) & 1) ^ 1, p.status);
+        const int mrow = m0 + kGmBM * static_cast<int>(rank);        // this CTA's A rows
+        const int nrow = n0 + Cfg::kBRows * static_cast<int>(rank);  // this CTA's B rows
+        for (int kt = 0; kt < slots && ok; ++kt, ++kt_global) {
+          const int s = kt_global % NS;
+          ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status);
           if (!ok) break;
+          const uint32_t fb = lead(bar_full(s));
+          auto load = [&](uint32_t dst, const CUtensorMap* m, int c0, int c1) {
+            if (kPair) tma_load_2d_pair(dst, m, fb, c0, c1);
+            else tma_load_2d(dst, m, fb, c0, c1);
+          };
           if (kt < ktiles) {
-            const int nkb = min(4, kblocks - 4 * kt);
-            mbar_arrive_expect_tx(bar_full(s), kGmAStage + kGmBStage + nkb * 512 * (1 + n_sfb));
-            tma_load_2d(a_st(s), &tm_a, bar_full(s), kt * kGmBKBytes, m0);
-            tma_load_2d(b_st(s), &tm_b, bar_full(s), kt * kGmBKBytes, n0);
-            bulk_load(sfa_st(s), p.a_scales + (static_cast<size_t>(mb) * kblocks + 4 * kt) * 512,
-                      nkb * 512, bar_full(s));
-            for (int j = 0; j < n_sfb; ++j)
-              bulk_load(sfb_st(s) + j * 2048,
-                        p.w_scales + (static_cast<size_t>(n0 / 128 + j) * kblocks + 4 * kt) * 512,
-                        nkb * 512, bar_full(s));
+            if (leader)
+              mbar_arrive_expect_tx(bar_full(s),
+                                    Cfg::kCtas * (kGmAStage + Cfg::kBStage + kGmSfaStage + kGmSfbStage));
+            load(a_st(s), &tm_a, kt * kGmBKBytes, mrow);
+            load(b_st(s), &tm_b, kt * kGmBKBytes, nrow);
+            // scale atoms viewed as rows of 256 B: 4 atoms = 8 rows
+            load(sfa_st(s), &tm_sfa, 0, ((mrow / 128) * kblocks + 4 * kt) * 2);
+            for (int j = 0; j < 2; ++j)
+              load(sfb_st(s) + j * 2048, &tm_sfb, 0, ((n0 / 128 + j) * kblocks + 4 * kt) * 2);
           } else {
-            // low-rank slot: L2 rows [32 c, 32 c + 32) x columns [n0, n0 + 256),
-            // four 64-wide boxes (rows past r read as zero)
+            // low-rank slot: L2 rows [32 c, 32 c + 32) x this CTA's columns, 64-wide
+            // boxes (rows past r read as zero)
             const int c = kt - ktiles;
-            mbar_arrive_expect_tx(bar_full(s), kGmLrBTile);
-            for (int nb = 0; nb < 4; ++nb)
-              tma_load_2d(stage(s) + nb * (kGmLrK * 128), &tm_l2, bar_full(s), n0 + nb * 64,
-                          c * kGmLrK);
+            if (leader) mbar_arrive_expect_tx(bar_full(s), kGmLrK * kGmBN * 2);
+            for (int nb = 0; nb < Cfg::kBRows / 64; ++nb)
+              load(stage(s) + nb * (kGmLrK * 128), &tm_l2, nrow + nb * 64, c * kGmLrK);
           }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
+    if (leader && elect_one()) {
       bool ok = true;
-      const uint32_t id_lr = idesc_bf16_f32(128, kGmBN, false, true);
+      const uint32_t mma_m = kGmBM * Cfg::kCtas;
+      const uint32_t id_lr = idesc_bf16_f32(mma_m, kGmBN, false, true);
+      const uint32_t id_fp4 = idesc_nvfp4(mma_m, kGmBN);
       int kt_global = 0;
       for (int i = 0; i < my_tiles && ok; ++i) {
-        int m0, n0;
-        tile_mn(i, m0, n0);
-        const int n_tile = min(kGmBN, p.N - n0);
-        const int n_sfb = n_tile > 128 ? 2 : 1;
         const uint32_t acc = tmem + ((i & 1) ? kTmAcc1 : 0u);
-        // the previous tile's epilogue has drained the overlapped columns
+        // the previous tile's epilogues (both CTAs) drained the overlapped columns
         if (i > 0) {
           ok = mbar_wait(bar_acc_free, (i - 1) & 1, p.status);
           if (!ok) break;
         }
         tc_fence_after();
-        const uint32_t id_fp4 = idesc_nvfp4(128, n_tile);
-        for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
-          const int s = kt_global % kGmStages;
-          ok = mbar_wait(bar_full(s), (kt_global / kGmStages) & 1, p.status);
+        for (int kt = 0; kt < slots && ok; ++kt, ++kt_global) {
+          const int s = kt_global % NS;
+          ok = mbar_wait(bar_full(s), (kt_global / NS) & 1, p.status);
           if (!ok) break;
           tc_fence_after();
           if (kt < ktiles) {
             const int nkb = min(4, kblocks - 4 * kt);
             for (int kb = 0; kb < nkb; ++kb) {
-              tc_cp_32x128b_warpx4(tmem + kTmSfa + 4 * kb,
-                                   smem_desc(sfa_st(s) + kb * 512, 128, 128, kSwizzleNone));
-              for (int j = 0; j < n_sfb; ++j)
-                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb + 4 * j,
-                                     smem_desc(sfb_st(s) + j * 2048 + kb * 512, 128, 128,
-                                               kSwizzleNone));
+              const uint64_t da = smem_desc(sfa_st(s) + kb * 512, 128, 128, kSwizzleNone);
+              const uint64_t db0 = smem_desc(sfb_st(s) + kb * 512, 128, 128, kSwizzleNone);
+              const uint64_t db1 = smem_desc(sfb_st(s) + 2048 + kb * 512, 128, 128, kSwizzleNone);
+              if (kPair) {
+                tc_cp_32x128b_warpx4_pair(tmem + kTmSfa + 4 * kb, da);
+                tc_cp_32x128b_warpx4_pair(tmem + kTmSfb + 8 * kb, db0);
+                tc_cp_32x128b_warpx4_pair(tmem + kTmSfb + 8 * kb + 4, db1);
+              } else {
+                tc_cp_32x128b_warpx4(tmem + kTmSfa + 4 * kb, da);
+                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb, db0);
+                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb + 4, db1);
+              }
             }
             for (int kb = 0; kb < nkb; ++kb) {
               const uint64_t ad = smem_desc(a_st(s) + kb * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(b_st(s) + kb * 32, 16, 1024, kSwizzle128B);
-              mma_nvfp4(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
-                        (kt > 0 || kb > 0) ? 1u : 0u);
+              const uint32_t accum = (kt > 0 || kb > 0) ? 1u : 0u;
+              if (kPair)
+                mma_nvfp4_pair(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
+                               accum);
+              else
+                mma_nvfp4(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
+                          accum);
             }
           } else {
             // low-rank slot: B = L2 chunk (MN-major, 128-byte swizzle; 64-wide N
             // blocks 4096 B apart = LBO, 8-deep K groups 1024 B apart = SBO);
             // A = xl1 hi / lo (no-swizzle K-major: K-adjacent core matrices 128 B
             // apart = LBO, 8-row groups 512 B apart = SBO)
-            const uint32_t a_hi = stage(s) + kGmLrBTile, a_lo = a_hi + kGmLrATile;
+            const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
 #pragma unroll
             for (int kk = 0; kk < kGmLrK / 16; ++kk) {
               const uint64_t bd = smem_desc(stage(s) + kk * 2048, kGmLrK * 128, 1024, kSwizzle128B);
-              mma_f16(acc, smem_desc(a_hi + kk * 256, 128, 512, kSwizzleNone), bd, id_lr, 1u);
-              mma_f16(acc, smem_desc(a_lo + kk * 256, 128, 512, kSwizzleNone), bd, id_lr, 1u);
+              const uint64_t ah = smem_desc(a_hi + kk * 256, 128, 512, kSwizzleNone);
+              const uint64_t al = smem_desc(a_lo + kk * 256, 128, 512, kSwizzleNone);
+              if (kPair) {
+                mma_f16_pair(acc, ah, bd, id_lr, 1u);
+                mma_f16_pair(acc, al, bd, id_lr, 1u);
+              } else {
+                mma_f16(acc, ah, bd, id_lr, 1u);
+                mma_f16(acc, al, bd, id_lr, 1u);
+              }
             }
           }
-          tc_commit(bar_empty(s));
+          if (kPair) tc_commit_pair(bar_empty(s), 0x3);
+          else tc_commit(bar_empty(s));
         }
-        tc_commit(bar_acc_full);
+        if (kPair) tc_commit_pair(bar_acc_full, 0x3);
+        else tc_commit(bar_acc_full);
       }
     }
   } else if (warp < 6) {
@@ -240,9 +273,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
-      const int m = m0 + trow;
-      for (int kt = 0; kt < ktiles + lr_chunks && ok; ++kt, ++kt_global) {
-        const int s = kt_global % kGmStages;
+      const int m = m0 + kGmBM * static_cast<int>(rank) + trow;
+      for (int kt = 0; kt < slots && ok; ++kt, ++kt_global) {
+        const int s = kt_global % NS;
         float v[kGmLrK];
         const int c = kt - ktiles;
         if (c >= 0) {
@@ -257,10 +290,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
           }
         }
-        ok = mbar_wait(bar_empty(s), ((kt_global / kGmStages) & 1) ^ 1, p.status);
+        ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status);
         if (!ok) break;
         if (c >= 0) {
-          const uint32_t a_hi = stage(s) + kGmLrBTile, a_lo = a_hi + kGmLrATile;
+          const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
 #pragma unroll
           for (int cm = 0; cm < kGmLrK / 8; ++cm) {
             uint32_t hi[4], lo[4];
@@ -284,7 +317,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_full(s));
+        if (lane == 0) {
+          if (kPair) mbar_arrive_cluster(lead(bar_full(s)));
+          else mbar_arrive(bar_full(s));
+        }
       }
     }
   } else {
@@ -295,14 +331,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     // the next tile's MMAs are let in after a single tensor-memory load per warp.
     const int quad = warp & 3;          // tensor-memory lanes 32 quad .. 32 quad + 31
     const int half = (warp - 6) >> 2;   // 0 or 1
-    const uint32_t out_buf = sbase + L.out + (warp - 6) * kGmStageOut;
-    float* bias_s = reinterpret_cast<float*>(smem + L.bias) + (warp - 6) * 128;  // [4][32]
+    const uint32_t out_buf = sbase + Cfg::kOut + (warp - 6) * kGmStageOut;
+    float* bias_s = reinterpret_cast<float*>(smem + Cfg::kBias) + (warp - 6) * 128;  // [4][32]
+    const uint32_t free_bar = lead(bar_acc_free);
     bool ok = true;
     int stores = 0;
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
-      const int n_tile = min(kGmBN, p.N - n0);
+      const int mrow = m0 + kGmBM * static_cast<int>(rank);
       const bool odd = i & 1;
       const uint32_t t_row = tmem + (odd ? kTmAcc1 : 0u) + (static_cast<uint32_t>(quad * 32) << 16);
       // sub-tile order: the overlapped one, then three of the six others
@@ -331,9 +368,12 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           // this warp's overlapped columns are in registers: let the next tile's MMAs in
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_acc_free);
+          if (lane == 0) {
+            if (kPair) mbar_arrive_cluster(free_bar);
+            else mbar_arrive(free_bar);
+          }
         }
-        if (j0 >= n_tile) continue;  // warp-uniform
+        if (n0 + j0 >= p.N || mrow >= p.M) continue;  // warp-uniform
         float y[32];
         const float4* bv = reinterpret_cast<const float4*>(bias_s + t * 32);
 #pragma unroll
@@ -376,7 +416,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tm_y, buf, n0 + j0, m0 + quad * 32);
+          tma_store_2d(&tm_y, buf, n0 + j0, mrow + quad * 32);
           bulk_commit();
         }
         ++stores;
@@ -386,10 +426,13 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  // both CTAs' tensor memory is written by the leader's MMAs: release it only
+  // once every warp of the pair is done
+  if (kPair) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmCols);
+    if (kPair) tmem_dealloc_pair(tmem, kTmCols);
+    else tmem_dealloc(tmem, kTmCols);
   }
 }
 
