@@ -28,6 +28,7 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   int gemm_pairs = 0;  // co-resident clusters of the CTA-pair GEMM
+  int gemm_pair_mode = -1;  // -1: by shape; SVDQ_GEMM_PAIR=0/1 forces single-CTA / CTA-pair tiles
   uint32_t* status = nullptr;
 };
 
@@ -104,6 +105,7 @@ svdq_status device_setup(DeviceInfo** out) {
         std::fprintf(stderr, "svdq: %d SMs, %d co-resident GEMM CTA pairs\n", d.num_sms,
                      d.gemm_pairs);
     }
+    if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) d.gemm_pair_mode = std::atoi(e) != 0;
     d.status = static_cast<uint32_t*>(st);
     d.ready = true;
   }
@@ -294,8 +296,11 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
 
-  // pairs of CTAs (cta_group::2, 256-row tiles) unless M fits one CTA's 128 rows
-  const bool pair = M > kGmBM;
+  // CTA pairs (cta_group::2, 256-row tiles) pay off only when the K loop is long
+  // enough to hide their cross-CTA barrier traffic: measured on B200, single
+  // CTAs win at K = 3072 (with or without the low-rank branch), pairs at K >= 8192.
+  const bool pair_auto = K >= 8192;
+  const bool pair = (d->gemm_pair_mode < 0 ? pair_auto : d->gemm_pair_mode != 0) && M > kGmBM;
   const int ctas = pair ? 2 : 1;
   const int b_rows = kGmBN / ctas;
   CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y;

@@ -24,8 +24,10 @@
 // Each tile is a sequence of ring slots: K/256 FP4 slots, then ceil(r/32)
 // low-rank slots holding an L2 chunk (by TMA) and the matching xl1 hi/lo tiles
 // (by the staging warps). A slot's "full" barrier (the leader's) counts the
-// leader's producer, whose expected bytes cover both CTAs' loads, and every
-// staging warp of the pair; the MMA commit frees the slot in both CTAs.
+// leader's producer, whose expected bytes cover both CTAs' loads; a low-rank
+// slot's operand tiles are announced on the slot's "ready" barrier (the
+// leader's) by every staging warp of the pair; the MMA commit frees the slot
+// in both CTAs.
 // Two 256-column accumulators share tensor memory with a 64-column overlap
 // ([0, 256) and [192, 448)); scale factors sit in [448, 496). The epilogue
 // drains the overlapped columns of a tile first and releases them, so the next
@@ -60,7 +62,7 @@ struct GmCfg {
   static constexpr uint32_t kOut = kStages * kStageBytes;     // 1024-aligned
   static constexpr uint32_t kBias = kOut + kGmEpiWarps * kGmStageOut;
   static constexpr uint32_t kBars = kBias + kGmEpiWarps * 128 * 4;
-  static constexpr uint32_t kTmemSlot = kBars + 8 * (2 * kStages + 2);
+  static constexpr uint32_t kTmemSlot = kBars + 8 * (3 * kStages + 2);
   static constexpr size_t kSmemBytes = kTmemSlot + 16 + 1024;
   static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert(kLrBTile + 2 * kGmLrATile <= kStageBytes, "a low-rank slot fits in a stage");
@@ -114,7 +116,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   auto sfb_st = [&](int s) { return sfa_st(s) + kGmSfaStage; };
   auto bar_full = [&](int s) { return sbase + Cfg::kBars + 8 * s; };
   auto bar_empty = [&](int s) { return sbase + Cfg::kBars + 8 * (NS + s); };
-  const uint32_t bar_acc_full = sbase + Cfg::kBars + 8 * (2 * NS);
+  auto bar_ready = [&](int s) { return sbase + Cfg::kBars + 8 * (2 * NS + s); };
+  const uint32_t bar_acc_full = sbase + Cfg::kBars + 8 * (3 * NS);
   const uint32_t bar_acc_free = bar_acc_full + 8;
   // the leader's copies of the pipeline barriers, as seen from this CTA
   auto lead = [&](uint32_t a) { return kPair ? map_peer_smem(a, 0) : a; };
@@ -122,7 +125,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_full(s), 1 + 4 * Cfg::kCtas);  // leader producer (with tx) + staging warps
+      mbar_init(bar_full(s), 1);                  // leader producer (with tx)
+      mbar_init(bar_ready(s), 4 * Cfg::kCtas);    // staging warps of a low-rank slot
       mbar_init(bar_empty(s), 1);
     }
     mbar_init(bar_acc_full, 1);
@@ -197,6 +201,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const uint32_t id_lr = idesc_bf16_f32(mma_m, kGmBN, false, true);
       const uint32_t id_fp4 = idesc_nvfp4(mma_m, kGmBN);
       int kt_global = 0;
+      uint32_t lr_uses = 0;  // bit s: parity of the low-rank uses of ring slot s so far
       for (int i = 0; i < my_tiles && ok; ++i) {
         const uint32_t acc = tmem + ((i & 1) ? kTmAcc1 : 0u);
         // the previous tile's epilogues (both CTAs) drained the overlapped columns
@@ -238,6 +243,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                           accum);
             }
           } else {
+            ok = mbar_wait(bar_ready(s), (lr_uses >> s) & 1u, p.status);
+            lr_uses ^= 1u << s;
+            if (!ok) break;
+            tc_fence_after();
             // low-rank slot: B = L2 chunk (MN-major, 128-byte swizzle; 64-wide N
             // blocks 4096 B apart = LBO, 8-deep K groups 1024 B apart = SBO);
             // A = xl1 hi / lo (no-swizzle K-major: K-adjacent core matrices 128 B
@@ -274,52 +283,52 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       int m0, n0;
       tile_mn(i, m0, n0);
       const int m = m0 + kGmBM * static_cast<int>(rank) + trow;
-      for (int kt = 0; kt < slots && ok; ++kt, ++kt_global) {
+      // FP4 slots need nothing from the staging warps, but their "empty" phases
+      // are still waited in order: a parity wait is only meaningful one phase
+      // at a time, so skipping ahead could pass a phase that has not come yet.
+      for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global)
+        ok = mbar_wait(bar_empty(kt_global % NS), ((kt_global / NS) & 1) ^ 1, p.status);
+      for (int c = 0; c < lr_chunks && ok; ++c, ++kt_global) {
         const int s = kt_global % NS;
+        // load before waiting: the global read overlaps the wait for the slot
         float v[kGmLrK];
-        const int c = kt - ktiles;
-        if (c >= 0) {
-          // load before waiting: the global read overlaps the wait for the slot
-          const float4* src = reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r +
-                                                              c * kGmLrK);
+        const float4* src = reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r +
+                                                            c * kGmLrK);
 #pragma unroll
-          for (int j = 0; j < kGmLrK / 4; ++j) {
-            // rows past M and columns past r (r % 32 == 16) contribute zeros
-            const float4 f = (m < p.M && c * kGmLrK + 4 * j < p.r) ? __ldg(src + j)
-                                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
-          }
+        for (int j = 0; j < kGmLrK / 4; ++j) {
+          // rows past M and columns past r (r % 32 == 16) contribute zeros
+          const float4 f = (m < p.M && c * kGmLrK + 4 * j < p.r) ? __ldg(src + j)
+                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
         }
         ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status);
         if (!ok) break;
-        if (c >= 0) {
-          const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
+        const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
 #pragma unroll
-          for (int cm = 0; cm < kGmLrK / 8; ++cm) {
-            uint32_t hi[4], lo[4];
+        for (int cm = 0; cm < kGmLrK / 8; ++cm) {
+          uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float x0 = v[8 * cm + 2 * j], x1 = v[8 * cm + 2 * j + 1];
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-              const float2 hf = __bfloat1622float2(hb);
-              const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-              hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
-              lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
-            }
-            const uint32_t off = (trow >> 3) * 512 + cm * 128 + (trow & 7) * 16;
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi + off), "r"(hi[0]),
-                         "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
-                         : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo + off), "r"(lo[0]),
-                         "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
-                         : "memory");
+          for (int j = 0; j < 4; ++j) {
+            const float x0 = v[8 * cm + 2 * j], x1 = v[8 * cm + 2 * j + 1];
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(hb);
+            const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+            hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
+            lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
           }
-          fence_proxy_async_smem();
+          const uint32_t off = (trow >> 3) * 512 + cm * 128 + (trow & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi + off), "r"(hi[0]),
+                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo + off), "r"(lo[0]),
+                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                       : "memory");
         }
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (kPair) mbar_arrive_cluster(lead(bar_full(s)));
-          else mbar_arrive(bar_full(s));
+          if (kPair) mbar_arrive_cluster(lead(bar_ready(s)));
+          else mbar_arrive(bar_ready(s));
         }
       }
     }
