@@ -38,6 +38,8 @@ SMALL = [
     # more tiles than SMs: every persistent CTA walks several tiles, both accumulators
     WL.custom_svdq("many_tiles", 2048, 512, 2816, 32, seed=18),
     WL.custom_svdq("many_tiles_r128", 2176, 256, 2560, 128, seed=19),
+    # K >= 8192 selects CTA-pair tiles (256 rows); M and N ragged in both halves
+    WL.custom_svdq("long_k_pair", 400, 8192, 528, 32, seed=20),
 ]
 
 
