@@ -18,7 +18,9 @@ INT4 scales (activations and weights), group-major
 
 NVFP4 / INT4 codes
     Plain: row-major, K contiguous, two codes per byte, element 2j in the low
-    nibble. The tiled form is the same bytes.
+    nibble (INT4 as two's complement). The tiled NVFP4 codes are the same bytes.
+    Tiled INT4 codes hold each value v in -7..7 as a sign-magnitude nibble:
+    8 + |v| if v < 0, else v; nibble order as in the plain form.
 
 AWQ qweight, MMA-fragment order
     N padded to 16 rows. For row block b = n // 16 and group g = k // 64 there
@@ -90,6 +92,25 @@ def tile_int4_scales(scales: np.ndarray) -> np.ndarray:
 def untile_int4_scales(tiled: np.ndarray, rows: int, K: int) -> np.ndarray:
     t = np.asarray(tiled, dtype=np.uint16).reshape(K // 64, pad_rows(rows))
     return t[:, :rows].view(np.float16).astype(np.float64).T.copy()
+
+
+# --------------------------------------------------------------- INT4 codes
+def tile_int4_codes(q: np.ndarray) -> np.ndarray:
+    """q [rows, K] integers in -7..7 -> tiled bytes [rows, K/2] (sign-magnitude nibbles)."""
+    q = np.asarray(q).astype(np.int16)
+    if np.any(np.abs(q) > 7):
+        raise ValueError("INT4 codes must lie in -7..7")
+    nib = np.where(q < 0, 8 - q, q).astype(np.uint8)  # 8 + |q| for negative q
+    return (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+
+
+def untile_int4_codes(tiled: np.ndarray) -> np.ndarray:
+    """Tiled bytes [rows, K/2] -> q [rows, K] int16."""
+    t = np.asarray(tiled, dtype=np.uint8)
+    nib = np.empty(t.shape[:-1] + (t.shape[-1] * 2,), dtype=np.int16)
+    nib[..., 0::2] = t & 0xF
+    nib[..., 1::2] = t >> 4
+    return np.where(nib >= 8, -(nib - 8), nib).astype(np.int16)
 
 
 # --------------------------------------------------------------- AWQ qweight
