@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(kQaThreads, 2)
           for (int j = 0; j < 16; ++j) {
             int v = __float2int_rn(__fmul_rn(xh[j], rcp));
             v = max(-7, min(7, v));
-            const uint32_t nib = static_cast<uint32_t>(v) & 0xFu;
+            // tiled INT4 codes are sign-magnitude nibbles
+            const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
             if (j < 8) code_lo |= nib << (4 * j);
             else code_hi |= nib << (4 * (j - 8));
           }

@@ -12,6 +12,7 @@
 
 #include "../../include/svdq.h"
 #include "awq.cuh"
+#include "int4_gemm.cuh"
 #include "pack.cuh"
 #include "quantize_act.cuh"
 #include "w4a4_gemm.cuh"
@@ -74,6 +75,9 @@ svdq_status device_setup(DeviceInfo** out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(GmCfg<true>::kSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kI4SmemBytes)) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
     if (cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(awq_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -115,8 +119,12 @@ svdq_status device_setup(DeviceInfo** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool debug_on() { return std::getenv("SVDQ_DEBUG") != nullptr; }
+
 svdq_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess && debug_on()) std::fprintf(stderr, "svdq: launch failed: %s\n", cudaGetErrorString(e));
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
 bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
@@ -126,9 +134,14 @@ bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint6
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "svdq: tensor map (dims %llu x %llu, box %u x %u) failed: %d\n",
+                 static_cast<unsigned long long>(inner), static_cast<unsigned long long>(outer),
+                 box_inner, box_outer, static_cast<int>(r));
+  return r == CUDA_SUCCESS;
 }
 
 bool rank_ok(int r) { return r == 0 || (r % 16 == 0 && r >= 16 && r <= 256); }
@@ -140,6 +153,49 @@ unsigned grid_for(size_t n, unsigned threads) {
   if (b < 1) b = 1;
   if (b > 65535u * 8u) b = 65535u * 8u;
   return static_cast<unsigned>(b);
+}
+
+// INT4 W4A4 GEMM (w4a4_int4_gemm_kernel): packed codes [rows, K/2] as 64-byte
+// boxes, group-major FP16 scales [K/64][rows padded to 128] as 2-group boxes.
+svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, const void* a_codes,
+                             const void* a_scales, const float* xl1, const void* w_codes,
+                             const void* w_scales, const void* L2, const void* bias, void* Y,
+                             int ldy, svdq_out out, cudaStream_t stream) {
+  CUtensorMap tm_a, tm_b, tm_sa, tm_sw, tm_l2;
+  const uint64_t G = static_cast<uint64_t>(K / 64);
+  if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 64, kI4BM,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 64, kI4BN,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_scales, pad128(M), G, pad128(M) * 2,
+                    128, 2, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w_scales, pad128(N), G, pad128(N) * 2,
+                    128, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ERR_CUDA;
+  if (r > 0) {
+    if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, N, r,
+                      static_cast<uint64_t>(N) * 2, 64, kI4LrK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l2 = tm_a;
+  }
+  I4Params p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.xl1 = xl1;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = Y;
+  p.ldy = ldy;
+  p.out_f32 = out == SVDQ_OUT_F32;
+  p.status = d->status;
+  p.tiles_m = (M + kI4BM - 1) / kI4BM;
+  p.tiles = p.tiles_m * ((N + kI4BN - 1) / kI4BN);
+  const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
+  w4a4_int4_gemm_kernel<<<grid, kI4Threads, kI4SmemBytes, stream>>>(tm_a, tm_b, tm_sa, tm_sw,
+                                                                     tm_l2, p);
+  return launch_status();
 }
 
 }  // namespace
@@ -292,9 +348,11 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
       !aligned16(Y) || (xl1 && !aligned16(xl1)) || (L2 && !aligned16(L2)) ||
       (bias && !aligned16(bias)) || (static_cast<size_t>(ldy) * esz) % 16)
     return SVDQ_ERR_ALIGNMENT;
-  if (format != SVDQ_NVFP4_G16) return SVDQ_ERR_UNSUPPORTED;
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  if (format == SVDQ_INT4_G64)
+    return launch_int4_gemm(d, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, Y,
+                            ldy, out, static_cast<cudaStream_t>(stream));
 
   // CTA pairs (cta_group::2, 256-row tiles) pay off only when the K loop is long
   // enough to hide their cross-CTA barrier traffic: measured on B200, single
@@ -428,8 +486,12 @@ svdq_status svdq_pack(svdq_pack_kind kind, svdq_format format, int rows, int K,
     if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
     if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
     const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
-    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(plain_codes),
-                                                     static_cast<uint4*>(tiled_codes), n16);
+    if (format == SVDQ_NVFP4_G16)
+      copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(plain_codes),
+                                                       static_cast<uint4*>(tiled_codes), n16);
+    else
+      int4_codes_kernel<<<grid_for(n16 * 16, T), T, 0, s>>>(
+          static_cast<const uint8_t*>(plain_codes), static_cast<uint8_t*>(tiled_codes), n16 * 16, 1);
     if (format == SVDQ_NVFP4_G16) {
       const size_t n = pad128(rows) * (K / 16);
       pack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
@@ -480,8 +542,12 @@ svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K
     if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
     if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
     const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
-    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(tiled_codes),
-                                                     static_cast<uint4*>(plain_codes), n16);
+    if (format == SVDQ_NVFP4_G16)
+      copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(tiled_codes),
+                                                       static_cast<uint4*>(plain_codes), n16);
+    else
+      int4_codes_kernel<<<grid_for(n16 * 16, T), T, 0, s>>>(
+          static_cast<const uint8_t*>(tiled_codes), static_cast<uint8_t*>(plain_codes), n16 * 16, 0);
     if (format == SVDQ_NVFP4_G16) {
       const size_t n = static_cast<size_t>(rows) * (K / 16);
       unpack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(

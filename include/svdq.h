@@ -66,9 +66,13 @@ const char* svdq_status_str(svdq_status status);
 int svdq_version(void);
 
 /*
- * Buffer sizes in bytes of the storage formats below. Codes are plain row-major
+ * Buffer sizes in bytes of the storage formats below. Codes are row-major
  * packed nibbles, K contiguous, element 2j in the low nibble, 2j+1 in the high
- * nibble (INT4 as two's complement): rows * K / 2 bytes.
+ * nibble: rows * K / 2 bytes. NVFP4 codes are E2M1 in both the plain and the
+ * tiled form. INT4 values (-7..7) are two's-complement nibbles in the plain
+ * form and sign-magnitude nibbles (8 + |v| for v < 0) in the tiled form, which
+ * the GEMM expands to 8-bit tensor-core operands with three logic operations
+ * per four codes.
  * Scales ("tiled"):
  *  - NVFP4: rows padded to 128; for row m and scale column j = k/16 the byte sits
  *    in 512-byte atom a = (m/128) * (K/64) + j/4 at offset
@@ -101,7 +105,7 @@ size_t awq_sz_bytes(int N, int K);
  * L1s        device, the down-projection operand from svdq_pack_lowrank: bf16
  *            [2][r][K] = diag(smooth_inv) L1, transposed, as hi and lo planes;
  *            NULL iff r == 0
- * codes      device, svdq_codes_bytes(format, M, K) bytes, written
+ * codes      device, svdq_codes_bytes(format, M, K) bytes, written (tiled form)
  * scales     device, svdq_scales_bytes(format, M, K) bytes, written (padding rows too)
  * xl1        device, float32 [M, r], written; NULL iff r == 0
  * Codes and scales are bit-exact functions of the inputs. xl1 is computed on the
@@ -130,6 +134,9 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
  * Y                  device, [M, ldy] bf16 (out = SVDQ_OUT_BF16) or float32, ldy >= N,
  *                    ldy * element size % 16 == 0
  * The low-rank product uses xl1 split into two bf16 terms; accumulation is float32.
+ * NVFP4 runs on the block-scaled FP4 MMA. INT4 has no integer 4-bit MMA on
+ * sm_100a: each 64-wide group's product is formed exactly on the tensor cores
+ * (codes as E4M3 values v/512) and scaled by s_a s_w on the CUDA cores.
  */
 svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
@@ -159,7 +166,9 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
  * svdq_pack / svdq_unpack -- convert between plain and tiled storage
  * (unpack(pack(x)) == x bit for bit).
  *
- * ACT / WEIGHT: plain_codes [rows, K/2] bytes -> tiled codes (the same bytes);
+ * ACT / WEIGHT: plain_codes [rows, K/2] bytes -> tiled codes (NVFP4: the same
+ *   bytes; INT4: two's complement -> sign-magnitude per nibble, where -8 is out
+ *   of contract);
  *   plain_scales: NVFP4 uint8 [rows, K/16] E4M3 codes, INT4 fp16 [rows, K/64]
  *   -> tiled scales (layouts above). plain_zeros must be NULL.
  * AWQ: plain_codes = qweight [N, K/2] (element 2j low nibble, values 0..15),

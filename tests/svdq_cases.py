@@ -45,6 +45,13 @@ def oracle_layer(shape: WL.SvdqShape, M: int | None = None) -> dict:
     return {"shape": shape, "x_bits": x_bits, "w_bits": d["W"], "bias_bits": d["bias"], **pr}
 
 
+def tiled_codes(fmt: str, q: np.ndarray) -> np.ndarray:
+    """Codes as the kernels store them: NVFP4 plain packed nibbles, INT4 sign-magnitude."""
+    if fmt == "nvfp4":
+        return S.pack_nibbles(q).reshape(-1)
+    return LO.tile_int4_codes(q).reshape(-1)
+
+
 def tiled_scales(fmt: str, scales: np.ndarray) -> np.ndarray:
     if fmt == "nvfp4":
         return LO.tile_nvfp4_scales(scales)

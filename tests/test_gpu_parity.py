@@ -42,6 +42,16 @@ SMALL = [
     WL.custom_svdq("long_k_pair", 400, 8192, 528, 32, seed=20),
 ]
 
+SMALL_INT4 = [
+    WL.custom_svdq("int4_ragged", 300, 640, 272, 32, fmt="int4", seed=16),
+    # an odd number of 64-wide groups (the last stage holds one) and r % 32 == 16
+    WL.custom_svdq("int4_odd_groups", 200, 576, 400, 16, fmt="int4", seed=24),
+    WL.custom_svdq("int4_one_row", 1, 128, 48, 16, fmt="int4", seed=25),
+    WL.custom_svdq("int4_r0", 130, 256, 160, 0, fmt="int4", seed=26),
+    WL.custom_svdq("int4_r256", 200, 512, 256, 256, fmt="int4", seed=27, spike_rank=8, spike_sv=5.0),
+    WL.custom_svdq("int4_many_tiles_r128", 2176, 256, 2560, 128, fmt="int4", seed=28),
+]
+
 
 def _quantize_gpu(bq, layer, X_bits, fmt, with_lowrank=True, smooth=True):
     X = C.bf16_tensor(X_bits)
@@ -53,15 +63,14 @@ def _quantize_gpu(bq, layer, X_bits, fmt, with_lowrank=True, smooth=True):
     return codes.cpu().numpy(), scales.cpu().numpy(), (xl1.cpu().numpy() if xl1 is not None else None)
 
 
-@pytest.mark.parametrize("shape", SMALL + [WL.custom_svdq("int4", 300, 640, 272, 32, fmt="int4", seed=16)],
-                         ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", SMALL + SMALL_INT4[:2], ids=lambda s: s.name)
 def test_quantize_act_matches_oracle(bq, shape):
     layer = C.oracle_layer(shape)
     x = F.bf16_from_bits(layer["x_bits"])
     xhat = S.smooth(x, layer["smooth_inv"])
     q, s = S.quantize(shape.fmt, xhat)
     codes, scales, xl1 = _quantize_gpu(bq, layer, layer["x_bits"], shape.fmt, shape.r > 0)
-    want_codes = S.pack_nibbles(q).reshape(-1)
+    want_codes = C.tiled_codes(shape.fmt, q)
     bad = np.nonzero(codes != want_codes)[0]
     assert bad.size == 0, f"{bad.size} code bytes differ, first at {bad[:5]}: {codes[bad[:5]]} vs {want_codes[bad[:5]]}"
     want_scales = C.tiled_scales(shape.fmt, s)
@@ -81,7 +90,7 @@ def test_weight_quantizer_mode(bq):
     for fmt in ("nvfp4", "int4"):
         codes, scales, _ = _quantize_gpu(bq, layer, R_bits, fmt, with_lowrank=False, smooth=False)
         q, s = S.quantize(fmt, layer["R"])
-        assert np.array_equal(codes, S.pack_nibbles(q).reshape(-1)), fmt
+        assert np.array_equal(codes, C.tiled_codes(fmt, q)), fmt
         assert np.array_equal(scales, C.tiled_scales(fmt, s)), fmt
 
 
@@ -106,7 +115,7 @@ def _gemm_inputs(layer, fmt):
     return xhat, qa, sa, xl1
 
 
-@pytest.mark.parametrize("shape", SMALL, ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", SMALL + SMALL_INT4, ids=lambda s: s.name)
 @pytest.mark.parametrize("with_bias", [True, False])
 def test_w4a4_linear_matches_oracle(bq, shape, with_bias):
     layer = C.oracle_layer(shape)
@@ -119,10 +128,10 @@ def test_w4a4_linear_matches_oracle(bq, shape, with_bias):
     ref = S.w4a4_linear(S.dequant(fmt, qa, sa), S.dequant(fmt, layer["w_codes"], layer["w_scales"]),
                         xl1, layer["L2"] if r else None, bias)
     args = dict(
-        a_codes=C.u8_tensor(S.pack_nibbles(qa).reshape(-1)),
+        a_codes=C.u8_tensor(C.tiled_codes(fmt, qa)),
         a_scales=C.u8_tensor(C.tiled_scales(fmt, sa)),
         xl1=C.f32_tensor(xl1) if r else None,
-        w_codes=C.u8_tensor(S.pack_nibbles(layer["w_codes"]).reshape(-1)),
+        w_codes=C.u8_tensor(C.tiled_codes(fmt, layer["w_codes"])),
         w_scales=C.u8_tensor(C.tiled_scales(fmt, layer["w_scales"])),
         L2=C.bf16_tensor(F.bf16_bits(layer["L2"])) if r else None,
         bias=C.bf16_tensor(layer["bias_bits"]) if with_bias else None,
@@ -159,21 +168,46 @@ def test_w4a4_exact_on_grid(bq):
     assert bad.size == 0, f"{len(bad)} outputs differ; first {bad[:4].tolist()}: {y[tuple(bad[0])]} vs {ref[tuple(bad[0])]}"
 
 
-def test_end_to_end_layer(bq):
+def test_w4a4_int4_exact_on_grid(bq):
+    """INT4 operands with power-of-two FP16 scales: every group's partial sum is
+    an exact integer, every scaled term and the float32 sum of the eight groups
+    fit in 24 bits, so the output must equal the oracle bit for bit. This pins
+    the code conversion, its K order, the scale placement and the exactness of
+    the tensor-core partial products."""
+    rng = np.random.default_rng(29)
+    M, Nn, K = 200, 272, 512
+    qa = rng.integers(-7, 8, size=(M, K))
+    qw = rng.integers(-7, 8, size=(Nn, K))
+    sa = 2.0 ** rng.integers(-2, 3, size=(M, K // 64))
+    sw = 2.0 ** rng.integers(-2, 3, size=(Nn, K // 64))
+    ref = S.w4a4_linear(S.dequant("int4", qa, sa), S.dequant("int4", qw, sw), None, None, None)
+    y = bq.svdq_w4a4_linear(C.u8_tensor(C.tiled_codes("int4", qa)),
+                            C.u8_tensor(C.tiled_scales("int4", sa)), None,
+                            C.u8_tensor(C.tiled_codes("int4", qw)),
+                            C.u8_tensor(C.tiled_scales("int4", sw)), None, None,
+                            M=M, N_=Nn, K=K, fmt="int4", out_dtype=torch.float32)
+    assert bq.svdq_check_device_status() == 0
+    y = y.cpu().numpy().astype(np.float64)
+    bad = np.argwhere(y != ref)
+    assert bad.size == 0, f"{len(bad)} outputs differ; first {bad[:4].tolist()}: {y[tuple(bad[0])]} vs {ref[tuple(bad[0])]}"
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_end_to_end_layer(bq, fmt):
     """quantize_act then w4a4_linear, against the oracle's whole forward."""
-    shape = WL.custom_svdq("e2e", 384, 1024, 512, 32, seed=22, n_outliers=8, outlier_scale=50.0,
-                           spike_rank=8, spike_sv=5.0)
+    shape = WL.custom_svdq("e2e", 384, 1024, 512, 32, fmt=fmt, seed=22, n_outliers=8,
+                           outlier_scale=50.0, spike_rank=8, spike_sv=5.0)
     layer = C.oracle_layer(shape)
-    fwd = S.svdq_forward("nvfp4", layer["x_bits"], layer["smooth_inv"], layer["L1"], layer["L2"],
+    fwd = S.svdq_forward(fmt, layer["x_bits"], layer["smooth_inv"], layer["L1"], layer["L2"],
                          layer["w_codes"], layer["w_scales"], layer["bias_bits"])
     X = C.bf16_tensor(layer["x_bits"])
     si = C.f32_tensor(layer["smooth_inv"])
     L1s = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si)
-    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si)
-    y = bq.svdq_w4a4_linear(codes, scales, xl1, C.u8_tensor(S.pack_nibbles(layer["w_codes"]).reshape(-1)),
-                            C.u8_tensor(LO.tile_nvfp4_scales(layer["w_scales"])),
+    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si, fmt=fmt)
+    y = bq.svdq_w4a4_linear(codes, scales, xl1, C.u8_tensor(C.tiled_codes(fmt, layer["w_codes"])),
+                            C.u8_tensor(C.tiled_scales(fmt, layer["w_scales"])),
                             C.bf16_tensor(F.bf16_bits(layer["L2"])), C.bf16_tensor(layer["bias_bits"]),
-                            M=shape.M, N_=shape.N, K=shape.K)
+                            M=shape.M, N_=shape.N, K=shape.K, fmt=fmt)
     assert bq.svdq_check_device_status() == 0
     C.assert_gemm_close(y.float().cpu().numpy().astype(np.float64), fwd["Y"], bf16_out=True)
 
@@ -193,7 +227,13 @@ def test_pack_lowrank_matches_oracle(bq, r, with_smooth):
 def test_pack_unpack_round_trip(bq, fmt):
     rng = np.random.default_rng(23)
     rows, K = 200, 384
-    codes = rng.integers(0, 256, size=rows * K // 2).astype(np.uint8)
+    if fmt == "nvfp4":
+        codes = rng.integers(0, 256, size=rows * K // 2).astype(np.uint8)
+        want_codes = codes
+    else:
+        q = rng.integers(-7, 8, size=(rows, K))
+        codes = S.pack_nibbles(q).reshape(-1)          # plain: two's complement
+        want_codes = C.tiled_codes("int4", q)          # tiled: sign-magnitude
     if fmt == "nvfp4":
         plain = rng.integers(0, 127, size=(rows, K // 16)).astype(np.uint8)
         want = LO.tile_nvfp4_scales(plain)
@@ -203,7 +243,7 @@ def test_pack_unpack_round_trip(bq, fmt):
         want = LO.tile_int4_scales(plain).view(np.uint8)
         plain_t = C.u8_tensor(plain.astype(np.float16).view(np.uint8).reshape(-1))
     tc, ts = bq.svdq_pack("weight", fmt, rows, K, C.u8_tensor(codes), plain_t)
-    assert np.array_equal(tc.cpu().numpy(), codes)
+    assert np.array_equal(tc.cpu().numpy(), want_codes)
     assert np.array_equal(ts.cpu().numpy(), want)
     pc = torch.empty_like(C.u8_tensor(codes))
     ps = torch.empty_like(plain_t)
@@ -294,6 +334,37 @@ def test_full_size_qkv_sampled(bq):
     assert np.all(np.abs(got_xl1 - ref_xl1) <= C.xl1_bound(xhat[rows], layer["L1"]))
     ref = S.w4a4_linear(S.dequant_nvfp4(q[rows], sc[rows]),
                         S.dequant_nvfp4(layer["w_codes"], layer["w_scales"]),
+                        S.down_proj(xhat[rows], layer["L1"]), layer["L2"],
+                        F.bf16_from_bits(layer["bias_bits"]))
+    C.assert_gemm_close(y.float().cpu().numpy()[rows].astype(np.float64), ref, bf16_out=True)
+
+
+@pytest.mark.slow
+def test_full_size_fc1_int4_sampled(bq):
+    """The FLUX-like fc1 layer in INT4 g64 at full size (M=4608, K=3072,
+    N=12288, r=128), weights quantized by the library: codes and scales
+    bit-exact, Y on sampled rows."""
+    shape = WL.FC1_INT4
+    layer = C.oracle_layer(shape)
+    x = F.bf16_from_bits(layer["x_bits"])
+    X = C.bf16_tensor(layer["x_bits"])
+    si = C.f32_tensor(layer["smooth_inv"])
+    L1s = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si)
+    wc, ws, _ = bq.svdq_quantize_act(C.bf16_tensor(F.bf16_bits(layer["R"])), None, None, fmt="int4")
+    codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si, fmt="int4")
+    y = bq.svdq_w4a4_linear(codes, scales, xl1, wc, ws, C.bf16_tensor(F.bf16_bits(layer["L2"])),
+                            C.bf16_tensor(layer["bias_bits"]), M=shape.M, N_=shape.N, K=shape.K,
+                            fmt="int4")
+    assert bq.svdq_check_device_status() == 0
+    assert np.array_equal(wc.cpu().numpy(), C.tiled_codes("int4", layer["w_codes"]))
+    assert np.array_equal(ws.cpu().numpy(), C.tiled_scales("int4", layer["w_scales"]))
+    xhat = S.smooth(x, layer["smooth_inv"])
+    q, sc = S.quantize_int4(xhat)
+    assert np.array_equal(codes.cpu().numpy(), C.tiled_codes("int4", q))
+    assert np.array_equal(scales.cpu().numpy(), C.tiled_scales("int4", sc))
+    rows = np.unique(np.concatenate([np.arange(0, shape.M, 131), [shape.M - 1]]))
+    ref = S.w4a4_linear(S.dequant("int4", q[rows], sc[rows]),
+                        S.dequant("int4", layer["w_codes"], layer["w_scales"]),
                         S.down_proj(xhat[rows], layer["L1"]), layer["L2"],
                         F.bf16_from_bits(layer["bias_bits"]))
     C.assert_gemm_close(y.float().cpu().numpy()[rows].astype(np.float64), ref, bf16_out=True)
