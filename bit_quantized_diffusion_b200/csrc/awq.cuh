@@ -18,27 +18,37 @@
 // bf16 pattern 0x4300 is the exact bf16 pair (128 + q), so the dequantization
 // is one mask per pair; the zero point enters once per group through xs.
 //
-// Each warp owns a contiguous run of groups of one 16-row block; its weights
-// and (scale, zero) pairs are two contiguous byte ranges, fetched by bulk
-// copies into shared memory so that every load of the CTA is in flight at once.
-// X is staged in shared memory once per CTA, rows 16 bytes longer than K so the
-// B-fragment reads of the 8 token rows fall in distinct banks.
+// Persistent: one CTA per SM streams a contiguous run of 16-row blocks. Its
+// producer warp bulk-copies each block's weights and (scale, zero) pairs (up
+// to 48 groups per ring stage; a block of more groups spans several stages)
+// through a ring in shared memory, starting at once; meanwhile the sixteen
+// consumer warps stage X and the token sums xs. X rows are 16 bytes longer
+// than K and, inside every 64-wide group, hold a lane's B fragments for the
+// group's four K steps as 32 contiguous bytes (lane quad t: words t and t + 4
+// of each 16-element step), so a lane reads them with two 16-byte loads and
+// the 8 token rows fall in distinct banks. Consumer warp w takes the w-th
+// sixteenth of every stage's groups, each group's four MMAs as two independent
+// accumulation chains. After a block's last stage each consumer drops its
+// partial sums into a slot of a small ring and moves on; a reducer warp adds
+// the sixteen partials of each block in a fixed order and writes Y, so no
+// consumer ever waits for another.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace svdq {
 
-constexpr int kAwqParts = 8;                 // warps sharing one 16-row block (K split)
-constexpr int kAwqBlocksPerCta = 2;          // 16-row blocks per CTA
-constexpr int kAwqWarps = kAwqParts * kAwqBlocksPerCta;
-constexpr int kAwqThreads = 32 * kAwqWarps;  // 512
-constexpr int kAwqBatch = 6;                 // groups per warp per bulk copy
-constexpr int kAwqGroupBytes = 512 + 64;     // fragment words + (s, z) pairs of 16 rows
+constexpr int kAwqConsumers = 16;                         // warps sharing each block (K split)
+constexpr int kAwqThreads = 32 * (kAwqConsumers + 2);     // + producer and reducer warps
+constexpr int kAwqRedSlots = 4;                           // blocks of partial sums in flight
+constexpr int kAwqStageGroups = 48;                       // groups per ring stage at most
+constexpr int kAwqGroupBytes = 512 + 64;                  // fragment words + (s, z) of 16 rows
+constexpr int kAwqMaxStages = 4;
 constexpr int kAwqMaxM = 64;
 
 struct AwqParams {
   int M, N, K;
+  int stages;             // ring depth (2..4)
   const __nv_bfloat16* X;
   const uint4* qweight;   // fragment order
   const uint32_t* sz;     // (s, z) bf16 pairs
@@ -47,58 +57,294 @@ struct AwqParams {
   uint32_t* status;
 };
 
-// dynamic shared memory: weight staging per warp, X rows, per-group token sums, barriers
-__host__ __device__ constexpr size_t awq_stage_bytes() {
-  return static_cast<size_t>(kAwqWarps) * kAwqBatch * kAwqGroupBytes;
+// dynamic shared memory: ring, X rows, token sums, reduction buffer, barriers
+__host__ __device__ constexpr int awq_stage_groups(int K) {
+  return K / 64 < kAwqStageGroups ? K / 64 : kAwqStageGroups;
+}
+__host__ __device__ constexpr size_t awq_stage_bytes(int K) {
+  return static_cast<size_t>(awq_stage_groups(K)) * kAwqGroupBytes;
 }
 __host__ __device__ constexpr size_t awq_xrow_bytes(int K) { return static_cast<size_t>(K) * 2 + 16; }
-__host__ __device__ constexpr size_t awq_smem_bytes(int M, int K) {
-  return awq_stage_bytes() + static_cast<size_t>(M + 1) * awq_xrow_bytes(K) +
-         static_cast<size_t>((M + 7) / 8) * 8 * (K / 64) * 4 + kAwqWarps * 8 + 128;
+__host__ __device__ constexpr size_t awq_fixed_bytes(int M, int K, int kMB) {
+  return static_cast<size_t>(M + 1) * awq_xrow_bytes(K) +               // X
+         static_cast<size_t>(kMB) * 8 * (K / 64) * 4 +                  // xs
+         static_cast<size_t>(kAwqRedSlots) * kAwqConsumers * 32 * 4 * kMB * 4 +  // partial sums
+         8 * 2 * (kAwqMaxStages + kAwqRedSlots) + 128;                  // barriers, alignment
+}
+__host__ __device__ constexpr size_t awq_smem_bytes(int M, int K, int kMB, int stages) {
+  return static_cast<size_t>(stages) * awq_stage_bytes(K) + awq_fixed_bytes(M, K, kMB);
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32"
       " {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float ldsf(uint32_t addr) { return __uint_as_float(lds32(addr)); }
+// The same with a compile-time byte offset folded into the instruction.
+template <int kOff>
+__device__ __forceinline__ uint4 lds128o(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr), "n"(kOff));
+  return v;
+}
+template <int kOff>
+__device__ __forceinline__ uint32_t lds32o(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(kOff));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// One fragment word (nibble s = bits 4s..4s+3) -> the four bf16 pairs
+// (128 + q[s], 128 + q[s + 4]), s = 0..3: even nibbles are gathered into the
+// bytes of `ev`, odd ones into `od`, and each pair is two byte selects next to
+// the exponent byte 0x43.
+__device__ __forceinline__ void awq_dequant_word(uint32_t w, uint32_t (&a)[4]) {
+  const uint32_t ev = w & 0x0F0F0F0Fu;
+  const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e43 = 0x43434343u;
+  a[0] = prmt(ev, e43, 0x4240u);  // nibbles 0, 4
+  a[1] = prmt(od, e43, 0x4240u);  // nibbles 1, 5
+  a[2] = prmt(ev, e43, 0x4341u);  // nibbles 2, 6
+  a[3] = prmt(od, e43, 0x4341u);  // nibbles 3, 7
+}
+
+// kN consecutive 64-wide groups of one warp: all shared-memory loads first,
+// then the groups' MMA chains (two per group: K steps 0, 1 and 2, 3)
+// interleaved, then the per-group scale and zero point.
+//   wp   this lane's first fragment word          (+512 per group)
+//   szp  (s, z) of row r0 of the first group        (+64 per group, row r0 + 8 at +32)
+//   xa   this lane's X fragment runs, xo the first group's offset in them (+128 per group)
+//   xsp  xs[c0][first group]                        (+4 per group, token c0 + 1 at +4 G)
+template <int kMB, int kN>  // kN <= 4
+__device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint32_t (&xa)[kMB],
+                                           uint32_t xo, uint32_t xsp, int G, float (&acc)[kMB][4]) {
+  uint4 w[kN], xl[kN][kMB][2];
+  uint32_t sz0[kN], sz8[kN];
+  float xs0[kN][kMB], xs1[kN][kMB];
+  uint32_t xb[kMB], xs0a[kMB], xs1a[kMB];
+#pragma unroll
+  for (int mb = 0; mb < kMB; ++mb) {
+    xb[mb] = xa[mb] + xo;
+    xs0a[mb] = xsp + mb * 8 * G * 4;
+    xs1a[mb] = xs0a[mb] + G * 4;
+  }
+#pragma unroll
+  for (int u = 0; u < kN; ++u) {
+    // u is a compile-time constant here: every offset below is an immediate
+    switch (u) {
+#define SVDQ_AWQ_LOADS(U)                                                        \
+  case U:                                                                        \
+    w[U] = lds128o<(U) * 512>(wp);                                               \
+    sz0[U] = lds32o<(U) * 64>(szp);                                              \
+    sz8[U] = lds32o<(U) * 64 + 32>(szp);                                         \
+    for (int mb = 0; mb < kMB; ++mb) {                                           \
+      xl[U][mb][0] = lds128o<(U) * 128>(xb[mb]);                                 \
+      xl[U][mb][1] = lds128o<(U) * 128 + 16>(xb[mb]);                            \
+      xs0[U][mb] = __uint_as_float(lds32o<(U) * 4>(xs0a[mb]));                   \
+      xs1[U][mb] = __uint_as_float(lds32o<(U) * 4>(xs1a[mb]));                   \
+    }                                                                            \
+    break;
+      SVDQ_AWQ_LOADS(0)
+      SVDQ_AWQ_LOADS(1)
+      SVDQ_AWQ_LOADS(2)
+      SVDQ_AWQ_LOADS(3)
+#undef SVDQ_AWQ_LOADS
+    }
+  }
+  float pc[kN][2][kMB][4];
+#pragma unroll
+  for (int u = 0; u < kN; ++u)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int mb = 0; mb < kMB; ++mb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pc[u][c][mb][e] = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+    for (int u = 0; u < kN; ++u) {
+      const uint32_t word = ks == 0 ? w[u].x : ks == 1 ? w[u].y : ks == 2 ? w[u].z : w[u].w;
+      uint32_t a[4];
+      awq_dequant_word(word, a);  // bf16 (128 + q) pairs
+#pragma unroll
+      for (int mb = 0; mb < kMB; ++mb) {
+        const uint4& x = xl[u][mb][ks >> 1];
+        mma_bf16_16816(pc[u][ks & 1][mb], a, (ks & 1) ? x.z : x.x, (ks & 1) ? x.w : x.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kN; ++u) {
+    const float s0 = __uint_as_float(sz0[u] << 16), s8 = __uint_as_float(sz8[u] << 16);
+    const float z0 = __uint_as_float(sz0[u] & 0xFFFF0000u) + 128.0f;
+    const float z8 = __uint_as_float(sz8[u] & 0xFFFF0000u) + 128.0f;
+#pragma unroll
+    for (int mb = 0; mb < kMB; ++mb) {
+      acc[mb][0] = fmaf(fmaf(-z0, xs0[u][mb], pc[u][0][mb][0] + pc[u][1][mb][0]), s0, acc[mb][0]);
+      acc[mb][1] = fmaf(fmaf(-z0, xs1[u][mb], pc[u][0][mb][1] + pc[u][1][mb][1]), s0, acc[mb][1]);
+      acc[mb][2] = fmaf(fmaf(-z8, xs0[u][mb], pc[u][0][mb][2] + pc[u][1][mb][2]), s8, acc[mb][2]);
+      acc[mb][3] = fmaf(fmaf(-z8, xs1[u][mb], pc[u][0][mb][3] + pc[u][1][mb][3]), s8, acc[mb][3]);
+    }
+  }
+}
+
 template <int kMB>  // number of 8-token blocks (1 or 2; the host splits larger M)
-__global__ void __launch_bounds__(kAwqThreads, 2) awq_gemv_kernel(const AwqParams p) {
+__global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~uintptr_t(127));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int blk = blockIdx.x * kAwqBlocksPerCta + warp / kAwqParts;  // 16-row block
-  const int part = warp % kAwqParts;
   const int G = p.K / 64;
-  const int g_begin = part * G / kAwqParts, g_end = (part + 1) * G / kAwqParts;
+  const int GS = awq_stage_groups(p.K);
+  const int nst = (G + GS - 1) / GS;                 // ring stages per block
+  const int NS = p.stages;
+  const size_t SB = awq_stage_bytes(p.K);
   const int nblocks = (p.N + 15) / 16;
+  const int b_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * nblocks / gridDim.x);
+  const int b_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * nblocks / gridDim.x);
   const int r0 = lane >> 2, c0 = 2 * (lane & 3);
 
-  uint8_t* wbuf = smem + static_cast<size_t>(warp) * kAwqBatch * kAwqGroupBytes;
+  uint8_t* ring = smem;
   const size_t xrow_bytes = awq_xrow_bytes(p.K);
-  uint8_t* xsm = smem + awq_stage_bytes();  // [M + 1][K + 8] bf16, row M all zero
+  uint8_t* xsm = ring + NS * SB;  // [M + 1][K + 8] bf16, row M all zero
   float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M + 1) * xrow_bytes);  // [kMB*8][G]
-  const uint32_t bar = smem_u32(xs + kMB * 8 * G) + warp * 8;
+  constexpr int kSlot = kAwqConsumers * 32 * 4 * kMB;  // floats per partial-sum slot
+  float* red = xs + kMB * 8 * G;                     // [slots][consumers][32][4 kMB]
+  const uint32_t bars = (smem_u32(red + kAwqRedSlots * kSlot) + 7) & ~7u;
+  auto full = [&](int s) { return bars + 8 * s; };
+  auto empty = [&](int s) { return bars + 8 * (kAwqMaxStages + s); };
+  auto red_full = [&](int q) { return bars + 8 * (2 * kAwqMaxStages + q); };
+  auto red_empty = [&](int q) { return bars + 8 * (2 * kAwqMaxStages + kAwqRedSlots + q); };
 
-  if (lane == 0) {
-    mbar_init(bar, 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), kAwqConsumers);
+    }
+    for (int q = 0; q < kAwqRedSlots; ++q) {
+      mbar_init(red_full(q), kAwqConsumers);
+      mbar_init(red_empty(q), 1);
+    }
     fence_barrier_init();
   }
-  // stage X in shared memory, plus one zero row that padding tokens read
-  for (int t = threadIdx.x; t < (p.M + 1) * (p.K / 8); t += kAwqThreads) {
-    const int m = t / (p.K / 8), c = t % (p.K / 8);
-    *reinterpret_cast<uint4*>(xsm + m * xrow_bytes + c * 16) =
-        m < p.M ? __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.K) + c)
-                : make_uint4(0u, 0u, 0u, 0u);
-  }
   __syncthreads();
+
+  if (warp == kAwqConsumers) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int b = b_begin; b < b_end && ok; ++b) {
+        for (int t = 0; t < nst && ok; ++t, ++it) {
+          const int s = it % NS;
+          // the producer and the reducer are not on the critical path: they
+          // wait suspended, leaving the issue slots to the consumers
+          ok = mbar_wait(empty(s), ((it / NS) & 1) ^ 1, p.status, kWaitLimitNs, 2000u);
+          if (!ok) break;
+          const int g0 = t * GS, n = min(GS, G - g0);
+          const size_t bg = static_cast<size_t>(b) * G + g0;
+          const uint32_t dst = smem_u32(ring + s * SB);
+          mbar_arrive_expect_tx(full(s), n * kAwqGroupBytes);
+          bulk_load(dst, p.qweight + bg * 32, n * 512, full(s));
+          bulk_load(dst + GS * 512, p.sz + bg * 16, n * 64, full(s));
+        }
+      }
+    }
+    return;  // the consumers synchronise among themselves from here on
+  }
+  if (warp == kAwqConsumers + 1) {
+    // ------------------------------------------------------------ reducer
+    for (int b = b_begin; b < b_end; ++b) {
+      const int jj = b - b_begin, q = jj % kAwqRedSlots;
+      const bool ok = mbar_wait(red_full(q), (jj / kAwqRedSlots) & 1, p.status, kWaitLimitNs, 2000u);
+      const float* rb = red + q * kSlot;
+#pragma unroll
+      for (int mb = 0; mb < kMB; ++mb) {
+        float4 v = *reinterpret_cast<const float4*>(rb + (lane * kMB + mb) * 4);
+#pragma unroll
+        for (int w = 1; w < kAwqConsumers; ++w) {
+          const float4 u = *reinterpret_cast<const float4*>(rb + ((w * 32 + lane) * kMB + mb) * 4);
+          v.x += u.x;
+          v.y += u.y;
+          v.z += u.z;
+          v.w += u.w;
+        }
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = b * 16 + r0 + ((j & 2) ? 8 : 0);
+          const int m = mb * 8 + c0 + (j & 1);
+          if (ok && n < p.N && m < p.M) {
+            const float bb = p.bias != nullptr ? __bfloat162float(p.bias[n]) : 0.0f;
+            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(vv[j] + bb);
+          }
+        }
+      }
+      __syncwarp();  // all lanes have read the slot
+      if (lane == 0) mbar_arrive(red_empty(q));
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  constexpr int kCT = kAwqConsumers * 32;
+  // X in shared memory, plus one zero row that padding tokens read. Source
+  // 16-byte unit c of a row holds words 4h..4h+3 (h = c % 2) of K step
+  // ks = (c / 2) % 4 of group c / 8; word 4h + t goes to lane quad t's run.
+  // Eight loads per thread are issued before any store, so their latencies overlap.
+  const int units = (p.M + 1) * (p.K / 8);
+  for (int t0 = threadIdx.x; t0 < units; t0 += 8 * kCT) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * kCT;
+      const int m = t / (p.K / 8), c = t % (p.K / 8);
+      v[u] = (t < units && m < p.M)
+                 ? __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.K) + c)
+                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * kCT;
+      if (t >= units) break;
+      const int m = t / (p.K / 8), c = t % (p.K / 8);
+      uint32_t* grp = reinterpret_cast<uint32_t*>(xsm + m * xrow_bytes + (c / 8) * 128);
+      const int ks = (c / 2) % 4, h = c % 2;
+      grp[0 * 8 + ks * 2 + h] = v[u].x;
+      grp[1 * 8 + ks * 2 + h] = v[u].y;
+      grp[2 * 8 + ks * 2 + h] = v[u].z;
+      grp[3 * 8 + ks * 2 + h] = v[u].w;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   // per-group token sums xs[m][g] (rows >= M are zero)
-  for (int t = threadIdx.x; t < kMB * 8 * G; t += kAwqThreads) {
+  for (int t = threadIdx.x; t < kMB * 8 * G; t += kCT) {
     const int m = t / G, g = t % G;
     float sum = 0.0f;
     if (m < p.M) {
@@ -114,98 +360,60 @@ __global__ void __launch_bounds__(kAwqThreads, 2) awq_gemv_kernel(const AwqParam
     }
     xs[t] = sum;
   }
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 
-  float acc[kMB][4];
+  // this lane's B-fragment runs: token rows r0 (+ 8 mb), lane quad t = lane % 4
+  // (rows >= M read the zero row)
+  uint32_t xa[kMB];
 #pragma unroll
-  for (int b = 0; b < kMB; ++b)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
-
-  if (blk < nblocks) {
-    // token rows this lane feeds as the B operand (rows >= M read the zero row)
-    const uint32_t* xrow[kMB];
-#pragma unroll
-    for (int b = 0; b < kMB; ++b) {
-      const int m = b * 8 + r0;
-      xrow[b] = reinterpret_cast<const uint32_t*>(xsm + (m < p.M ? m : p.M) * xrow_bytes) + c0 / 2;
-    }
-    uint32_t phase = 0;
-    for (int g0 = g_begin; g0 < g_end; g0 += kAwqBatch) {
-      const int ng = min(kAwqBatch, g_end - g0);
-      if (lane == 0) {
-        // one bulk copy each for the run's fragment words and its (s, z) pairs
-        mbar_arrive_expect_tx(bar, ng * kAwqGroupBytes);
-        bulk_load(smem_u32(wbuf), p.qweight + (static_cast<size_t>(blk) * G + g0) * 32, ng * 512,
-                  bar);
-        bulk_load(smem_u32(wbuf) + kAwqBatch * 512, p.sz + (static_cast<size_t>(blk) * G + g0) * 16,
-                  ng * 64, bar);
-      }
-      if (!mbar_wait(bar, phase, p.status)) break;
-      phase ^= 1;
-      const uint4* wq = reinterpret_cast<const uint4*>(wbuf) + lane;
-      const uint32_t* szs = reinterpret_cast<const uint32_t*>(wbuf + kAwqBatch * 512) + r0;
-#pragma unroll
-      for (int j = 0; j < kAwqBatch; ++j) {
-        if (j < ng) {
-          const int g = g0 + j;
-          const uint4 w = wq[j * 32];
-          const uint32_t sz0 = szs[j * 16], sz8 = szs[j * 16 + 8];
-          float part_acc[kMB][4];
-#pragma unroll
-          for (int b = 0; b < kMB; ++b)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) part_acc[b][e] = 0.0f;
-          const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a[4];
-#pragma unroll
-            for (int pr = 0; pr < 4; ++pr)
-              a[pr] = ((words[ks] >> (4 * pr)) & 0x000F000Fu) | 0x43004300u;  // bf16 (128 + q) pairs
-            const int kw = (g * 64 + ks * 16) / 2;  // 32-bit word index of the fragment
-#pragma unroll
-            for (int b = 0; b < kMB; ++b) mma_bf16_16816(part_acc[b], a, xrow[b][kw], xrow[b][kw + 4]);
-          }
-          const float s0 = __uint_as_float(sz0 << 16), s8 = __uint_as_float(sz8 << 16);
-          const float z0 = __uint_as_float(sz0 & 0xFFFF0000u) + 128.0f;
-          const float z8 = __uint_as_float(sz8 & 0xFFFF0000u) + 128.0f;
-#pragma unroll
-          for (int b = 0; b < kMB; ++b) {
-            const float xs0 = xs[(b * 8 + c0) * G + g], xs1 = xs[(b * 8 + c0 + 1) * G + g];
-            acc[b][0] = fmaf(fmaf(-z0, xs0, part_acc[b][0]), s0, acc[b][0]);
-            acc[b][1] = fmaf(fmaf(-z0, xs1, part_acc[b][1]), s0, acc[b][1]);
-            acc[b][2] = fmaf(fmaf(-z8, xs0, part_acc[b][2]), s8, acc[b][2]);
-            acc[b][3] = fmaf(fmaf(-z8, xs1, part_acc[b][3]), s8, acc[b][3]);
-          }
-        }
-      }
-      __syncwarp();  // every lane is done with the staging buffer before it is refilled
-    }
+  for (int mb = 0; mb < kMB; ++mb) {
+    const int m = mb * 8 + r0;
+    xa[mb] = smem_u32(xsm) + (m < p.M ? m : p.M) * static_cast<uint32_t>(xrow_bytes) + (lane & 3) * 32;
   }
-  // the first warp of each block adds the other K parts (in a fixed order) and
-  // writes Y, one 8-token block at a time, through the (now idle) staging memory
-  float* red = reinterpret_cast<float*>(smem);  // [kAwqWarps][32][4]
+  const uint32_t xs_a = smem_u32(xs) + c0 * G * 4;  // xs[c0][0]
+  bool ok = true;
+  int s = 0;          // ring slot
+  uint32_t ph = 0;    // its phase parity
+  for (int b = b_begin; b < b_end; ++b) {
+    float acc[kMB][4];
 #pragma unroll
-  for (int b = 0; b < kMB; ++b) {
-    __syncthreads();
+    for (int mb = 0; mb < kMB; ++mb)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) red[(warp * 32 + lane) * 4 + j] = acc[b][j];
-    __syncthreads();
-    if (part == 0 && blk < nblocks) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float v = red[(warp * 32 + lane) * 4 + j];
-#pragma unroll
-        for (int q = 1; q < kAwqParts; ++q) v += red[((warp + q) * 32 + lane) * 4 + j];
-        const int n = blk * 16 + r0 + ((j & 2) ? 8 : 0);
-        const int m = b * 8 + c0 + (j & 1);
-        if (n < p.N && m < p.M) {
-          const float bb = p.bias != nullptr ? __bfloat162float(p.bias[n]) : 0.0f;
-          p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(v + bb);
+      for (int j = 0; j < 4; ++j) acc[mb][j] = 0.0f;
+    for (int t = 0; t < nst; ++t) {
+      if (ok) ok = mbar_wait_poll(full(s), ph, p.status);
+      const int g0 = t * GS, n = min(GS, G - g0);
+      const int lo = warp * n / kAwqConsumers, hi = (warp + 1) * n / kAwqConsumers;
+      const uint32_t st = smem_u32(ring + s * SB);
+      const uint32_t wp = st + lo * 512 + lane * 16;           // this lane's fragment word
+      const uint32_t szp = st + GS * 512 + lo * 64 + r0 * 4;   // (s, z) of row r0
+      const uint32_t xo = (g0 + lo) * 128;                     // group offset in the X runs
+      const uint32_t xsp = xs_a + (g0 + lo) * 4;               // xs[c0][g]
+      if (ok) {
+        if (kMB == 1 && hi - lo == 3) {
+          awq_groups<kMB, 3>(wp, szp, xa, xo, xsp, G, acc);   // 48-group stages: 3 per warp
+        } else {
+          for (int j = 0; j < hi - lo; ++j)
+            awq_groups<kMB, 1>(wp + j * 512, szp + j * 64, xa, xo + j * 128, xsp + j * 4, G, acc);
         }
       }
+      __syncwarp();  // every lane is done with the stage before it is released
+      if (lane == 0) mbar_arrive(empty(s));
+      if (++s == NS) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
+    // hand this warp's partial sums of the block to the reducer
+    const int jj = b - b_begin, q = jj % kAwqRedSlots;
+    if (ok) ok = mbar_wait_poll(red_empty(q), ((jj / kAwqRedSlots) & 1) ^ 1, p.status);
+    float* rb = red + q * kSlot;
+#pragma unroll
+    for (int mb = 0; mb < kMB; ++mb)
+      *reinterpret_cast<float4*>(rb + ((warp * 32 + lane) * kMB + mb) * 4) =
+          make_float4(acc[mb][0], acc[mb][1], acc[mb][2], acc[mb][3]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(red_full(q));
   }
 }
 

@@ -92,11 +92,40 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Waits for the phase with the given parity to complete. Gives up after
 // `limit_ns` of global time: sets the timeout bit in *status and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_ns = kWaitLimitNs,
+                                          uint32_t hint_ns = 100000u) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+    if (global_ns() - t0 > limit_ns) {
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Polling form of mbar_wait: test_wait never suspends the thread, so a waiter
+// resumes as soon as the phase completes. Same time bound and status report.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, uint32_t* status,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
     if (global_ns() - t0 > limit_ns) {
       atomicOr(status, kStatusTimeout);
       return false;

@@ -434,28 +434,36 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
   // tokens per launch: at most 16 (two 8-token MMA blocks), and as many X rows
-  // as fit in shared memory beside the weight staging
+  // as fit in shared memory beside a weight ring of at least two stages
   const size_t smem_cap = 232448;
+  auto fits = [&](int mc, int stages) {
+    return awq_smem_bytes(mc, K, mc > 8 ? 2 : 1, stages) <= smem_cap;
+  };
   int mc = M < 16 ? M : 16;
-  while (mc > 1 && awq_smem_bytes(mc, K) > smem_cap) --mc;
-  if (awq_smem_bytes(mc, K) > smem_cap) return SVDQ_ERR_UNSUPPORTED;
+  while (mc > 1 && !fits(mc, 2)) --mc;
+  if (!fits(mc, 2)) return SVDQ_ERR_UNSUPPORTED;
   const int nblocks = (N + 15) / 16;
-  dim3 grid((nblocks + kAwqBlocksPerCta - 1) / kAwqBlocksPerCta);
+  // one persistent CTA per SM, each streaming a contiguous run of 16-row blocks
+  const int grid = nblocks < d->num_sms ? nblocks : d->num_sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int m0 = 0; m0 < M; m0 += mc) {
     const int mm = M - m0 < mc ? M - m0 : mc;
+    const int kmb = mm > 8 ? 2 : 1;
+    int stages = kAwqMaxStages;
+    while (stages > 2 && awq_smem_bytes(mm, K, kmb, stages) > smem_cap) --stages;
     AwqParams p;
     p.M = mm;
     p.N = N;
     p.K = K;
+    p.stages = stages;
     p.X = static_cast<const __nv_bfloat16*>(X) + static_cast<size_t>(m0) * K;
     p.qweight = static_cast<const uint4*>(qweight);
     p.sz = static_cast<const uint32_t*>(sz);
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.Y = static_cast<__nv_bfloat16*>(Y) + static_cast<size_t>(m0) * N;
     p.status = d->status;
-    const size_t smem = awq_smem_bytes(mm, K);
-    if (mm <= 8)
+    const size_t smem = awq_smem_bytes(mm, K, kmb, stages);
+    if (kmb == 1)
       awq_gemv_kernel<1><<<grid, kAwqThreads, smem, s>>>(p);
     else
       awq_gemv_kernel<2><<<grid, kAwqThreads, smem, s>>>(p);
