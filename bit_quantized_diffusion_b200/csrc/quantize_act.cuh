@@ -14,22 +14,23 @@
 // cluster of `ksplit` CTAs covers all of K for the same 128 rows; their partial
 // sums are added through distributed shared memory in a fixed order.
 //
-// Warp roles (18 warps):
+// Warp roles (10 warps):
 //   warp 0      TMA producer: X chunk [128 x 64] bf16 (128-byte swizzle), the L1s
 //               hi and lo chunks [r x 64] bf16, and 64 smooth_inv values
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
-//   warps 2..17 quantizers; warp q handles rows 8q..8q+7, lane l handles row
-//               8q + l%8 and columns 16(l/8)..16(l/8)+15 of the chunk: exactly one
-//               NVFP4 group (a quarter of an INT4 group)
+//   warps 2..9  quantizers; warp q handles rows 16q..16q+15, lane l handles row
+//               16q + l%16 and columns 32(l/16)..32(l/16)+31 of the chunk: two
+//               NVFP4 groups, or half an INT4 group (the other half is lane l^16);
+//               the float32 arithmetic runs on paired (f32x2) instructions
 #pragma once
 
 #include "sm100.cuh"
 
 namespace svdq {
 
-constexpr int kQaWarps = 18;
+constexpr int kQaWarps = 10;
 constexpr int kQaThreads = kQaWarps * 32;
-constexpr int kQaQuantWarps = 16;
+constexpr int kQaQuantWarps = 8;
 constexpr int kQaChunk = 64;                        // columns per stage
 constexpr int kQaXStageBytes = 128 * kQaChunk * 2;  // 16 KB
 constexpr int kQaSmoothBytes = kQaChunk * 4;        // 256 B
@@ -69,7 +70,7 @@ __host__ inline size_t qa_smem_bytes(int r, int stages) {
 }
 
 template <int kFmt>  // 0: NVFP4 (E2M1, UE4M3 per 16), 1: INT4 (FP16 per 64)
-__global__ void __launch_bounds__(kQaThreads, 2)
+__global__ void __launch_bounds__(kQaThreads, 3)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_l1, const QuantActParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -168,8 +169,8 @@ __global__ void __launch_bounds__(kQaThreads, 2)
   } else {
     // ---------------------------------------------------------------- quantizers
     const int qw = warp - 2;
-    const int row = qw * 8 + (lane & 7);
-    const int q = lane >> 3;  // which 16 columns of the chunk
+    const int row = qw * 16 + (lane & 15);
+    const int half = lane >> 4;  // which 32 columns of the chunk
     const int m = rb * 128 + row;
     const bool row_ok = m < p.M;
     bool ok = true;
@@ -178,92 +179,106 @@ __global__ void __launch_bounds__(kQaThreads, 2)
       const int kc = kc0 + i;
       ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status);
       if (!ok) break;
-      // -- 16 bf16 of this row from the 128B-swizzled X tile
-      float xh[16];
+      // -- 32 bf16 of this row from the 128B-swizzled X tile, as float32 pairs
+      uint64_t xp[16];
       {
         const uint32_t rowbase = x_stage(s) + row * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c = 2 * q + h;
+        for (int h = 0; h < 4; ++h) {
+          const int c = 4 * half + h;
           uint32_t v0, v1, v2, v3;
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
                        : "r"(rowbase + ((c ^ (row & 7)) << 4)));
           const uint32_t w[4] = {v0, v1, v2, v3};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            xh[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
-            xh[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-          }
+          for (int j = 0; j < 4; ++j)
+            xp[4 * h + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
         }
       }
       // -- a1: smoothing, one float32 multiply per element
       if (smoothing) {
         const float4* sp = reinterpret_cast<const float4*>(smem + (x_stage(s) - sbase) + L.sm_off) +
-                           4 * q;
+                           8 * half;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const float4 sv = sp[j];
-          xh[4 * j + 0] = __fmul_rn(xh[4 * j + 0], sv.x);
-          xh[4 * j + 1] = __fmul_rn(xh[4 * j + 1], sv.y);
-          xh[4 * j + 2] = __fmul_rn(xh[4 * j + 2], sv.z);
-          xh[4 * j + 3] = __fmul_rn(xh[4 * j + 3], sv.w);
+          xp[2 * j] = f2_mul(xp[2 * j], f2_pack(sv.x, sv.y));
+          xp[2 * j + 1] = f2_mul(xp[2 * j + 1], f2_pack(sv.z, sv.w));
         }
       }
       // this warp no longer reads the stage's shared memory
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty(s));
       // -- a2 + a3: group scale and codes
-      float amax = 0.0f;
+      float xh[32];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[j]));
-      uint32_t code_lo = 0, code_hi = 0;
+      for (int j = 0; j < 16; ++j) {
+        const float2 v = f2_unpack(xp[j]);
+        xh[2 * j] = v.x;
+        xh[2 * j + 1] = v.y;
+      }
+      uint32_t code[4];
       if (kFmt == 0) {
-        const uint32_t sc = e4m3_code(__fdiv_rn(amax, 6.0f));
-        const float2 vr = table[sc];  // (decoded scale, its reciprocal)
-        float y0[8], y1[8];
+        uint32_t sc[2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          y0[j] = __fmul_rn(xh[j], vr.y);
-          y1[j] = __fmul_rn(xh[8 + j], vr.y);
+        for (int g = 0; g < 2; ++g) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[16 * g + j]));
+          sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
+          const float2 vr = table[sc[g]];  // (decoded scale, its reciprocal)
+          const uint64_t rcp2 = f2_pack(vr.y, vr.y);
+          float y0[8], y1[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = f2_unpack(f2_mul(xp[8 * g + j], rcp2));
+            const float2 b = f2_unpack(f2_mul(xp[8 * g + 4 + j], rcp2));
+            y0[2 * j] = a.x;
+            y0[2 * j + 1] = a.y;
+            y1[2 * j] = b.x;
+            y1[2 * j + 1] = b.y;
+          }
+          const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
+          code[2 * g] = live ? e2m1x8(y0) : 0u;
+          code[2 * g + 1] = live ? e2m1x8(y1) : 0u;
         }
-        const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
-        code_lo = live ? e2m1x8(y0) : 0u;
-        code_hi = live ? e2m1x8(y1) : 0u;
-        // gather the row's four scale bytes into one word (lanes l, l+8, l+16, l+24)
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sc, 8);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sc, 16);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sc, 24);
-        if (q == 0) {
-          const uint32_t word = sc | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        // the row's four scale bytes: groups 2 half, 2 half + 1 here, the others in lane ^ 16
+        const uint32_t mine = sc[0] | (sc[1] << 8);
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
+        if (half == 0) {
+          const uint32_t word = mine | (other << 16);
           const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
           *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
               word;
         }
       } else {
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xh[j]));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
         const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
         const float sval = __half2float(hs);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) code[w] = 0u;
         if (sval != 0.0f) {
           const float rcp = __frcp_rn(sval);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 32; ++j) {
             int v = __float2int_rn(__fmul_rn(xh[j], rcp));
             v = max(-7, min(7, v));
             // tiled INT4 codes are sign-magnitude nibbles
             const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
-            if (j < 8) code_lo |= nib << (4 * j);
-            else code_hi |= nib << (4 * (j - 8));
+            code[j >> 3] |= nib << (4 * (j & 7));
           }
         }
-        if (q == 0)
+        if (half == 0)
           reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] =
               hs;
       }
       if (row_ok) {
-        *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + q * 8) =
-            make_uint2(code_lo, code_hi);
+        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + half * 16) =
+            make_uint4(code[0], code[1], code[2], code[3]);
       }
     }
     // ------------------------------------------------------------ xl1 epilogue
@@ -273,9 +288,9 @@ __global__ void __launch_bounds__(kQaThreads, 2)
     if (r > 0 && ok && mbar_wait(bar_acc, 0, p.status)) {
       tc_fence_after();
       const int quad = warp & 3;         // tensor-memory lanes this warp may read
-      const int part = (warp - 2) >> 2;  // which quarter of the r columns
+      const int part = (warp - 2) >> 2;  // which half of the r columns
       const int trow = quad * 32 + lane;
-      const int ncol = r / 4, c_begin = part * ncol;
+      const int ncol = r / 2, c_begin = part * ncol;
       const int rs = r + 4;  // padded row stride (floats) of the reduction buffer
       float* red = reinterpret_cast<float*>(smem + L.ring);
       const int tm = rb * 128 + trow;

@@ -78,6 +78,18 @@ svdq_status device_setup(DeviceInfo** out) {
     if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kI4SmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
+    // all of the SM's unified L1/shared storage as shared memory, so that the
+    // occupancy the host code plans for (e.g. two quantizer CTAs per SM) is real
+    for (const void* f : {reinterpret_cast<const void*>(quantize_act_kernel<0>),
+                          reinterpret_cast<const void*>(quantize_act_kernel<1>),
+                          reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<false>),
+                          reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true>),
+                          reinterpret_cast<const void*>(w4a4_int4_gemm_kernel),
+                          reinterpret_cast<const void*>(awq_gemv_kernel<1>),
+                          reinterpret_cast<const void*>(awq_gemv_kernel<2>)})
+      if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return SVDQ_ERR_CUDA;
     if (cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(awq_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -296,9 +308,20 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   const int per_sm = two_per_sm ? 2 : 1;
   const size_t smem_bytes = qa_smem_bytes(r, stages);
   auto kern = format == SVDQ_NVFP4_G16 ? quantize_act_kernel<0> : quantize_act_kernel<1>;
-  if (std::getenv("SVDQ_DEBUG") != nullptr)
-    std::fprintf(stderr, "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d\n",
-                 M, K, r, stages, per_sm, ksplit, ksplit * row_blocks);
+  if (debug_on()) {
+    int occ = -1;
+    (void)cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kQaThreads, smem_bytes);
+    cudaFuncAttributes fa;
+    (void)cudaFuncGetAttributes(&fa, kern);
+    std::fprintf(stderr,
+                 "  regs=%d static_smem=%zu max_dyn=%d carveout=%d local=%zu avail_dyn_for_2=%zu\n",
+                 fa.numRegs, fa.sharedSizeBytes, fa.maxDynamicSharedSizeBytes,
+                 fa.preferredShmemCarveout, fa.localSizeBytes, avail2);
+    std::fprintf(stderr,
+                 "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d smem=%zu "
+                 "occupancy=%d\n",
+                 M, K, r, stages, per_sm, ksplit, ksplit * row_blocks, smem_bytes, occ);
+  }
 
   QuantActParams p;
   p.M = M;
