@@ -311,12 +311,6 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   if (debug_on()) {
     int occ = -1;
     (void)cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kQaThreads, smem_bytes);
-    cudaFuncAttributes fa;
-    (void)cudaFuncGetAttributes(&fa, kern);
-    std::fprintf(stderr,
-                 "  regs=%d static_smem=%zu max_dyn=%d carveout=%d local=%zu avail_dyn_for_2=%zu\n",
-                 fa.numRegs, fa.sharedSizeBytes, fa.maxDynamicSharedSizeBytes,
-                 fa.preferredShmemCarveout, fa.localSizeBytes, avail2);
     std::fprintf(stderr,
                  "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d smem=%zu "
                  "occupancy=%d\n",
