@@ -330,7 +330,7 @@ def main() -> None:
     M, K, N, r = SHAPE.M, SHAPE.K, SHAPE.N, SHAPE.r
     codes = torch.empty(bq.svdq_codes_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
     scales = torch.empty(bq.svdq_scales_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
-    xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
+    xl1 = torch.empty((bq.svdq_xl1_splits(M, K, r), M, r), dtype=torch.float32, device=dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     Ya = torch.empty((AWQ.M, AWQ.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

@@ -58,12 +58,19 @@ def awq_sz_bytes(Nrows: int, K: int) -> int:
     return N.load().awq_sz_bytes(Nrows, K)
 
 
+def svdq_xl1_splits(M: int, K: int, r: int) -> int:
+    """S: svdq_quantize_act's xl1 buffer holds S x M x r float32 (its working space)."""
+    return N.load().svdq_xl1_splits(M, K, r)
+
+
 def svdq_quantize_act(X: torch.Tensor, L1s: torch.Tensor | None = None,
                       smooth_inv: torch.Tensor | None = None, fmt="nvfp4",
                       codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
                       xl1: torch.Tensor | None = None, stream=None):
     """Steps a1..a4 on X [M, K] bf16. L1s is the [2, r, K] bf16 operand from
-    svdq_pack_lowrank. Returns (codes, scales, xl1 or None)."""
+    svdq_pack_lowrank. xl1, if given, is a float32 buffer of at least
+    svdq_xl1_splits(M, K, r) * M * r elements (the call's working space).
+    Returns (codes, scales, xl1 [M, r] or None), xl1 a view of the buffer's start."""
     lib = N.load()
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bf16 tensor")
@@ -75,20 +82,21 @@ def svdq_quantize_act(X: torch.Tensor, L1s: torch.Tensor | None = None,
         codes = torch.empty(lib.svdq_codes_bytes(f, M, K), dtype=torch.uint8, device=dev)
     if scales is None:
         scales = torch.empty(lib.svdq_scales_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    S = lib.svdq_xl1_splits(M, K, r) if r else 0
     if r and xl1 is None:
-        xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
+        xl1 = torch.empty((S, M, r), dtype=torch.float32, device=dev)
     _need(codes, lib.svdq_codes_bytes(f, M, K), "codes")
     _need(scales, lib.svdq_scales_bytes(f, M, K), "scales")
     if L1s is not None and (L1s.dtype != torch.bfloat16 or tuple(L1s.shape) != (2, r, K)):
         raise ValueError("L1s must be bf16 [2, r, K]")
     if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
         raise ValueError("smooth_inv must be float32 [K]")
-    if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < M * r):
-        raise ValueError("xl1 must be float32 [M, r]")
+    if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < S * M * r):
+        raise ValueError(f"xl1 must be float32 [{S}, M, r]")
     N.check(lib.svdq_quantize_act(f, M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(L1s),
                                   _ptr(codes), _ptr(scales), _ptr(xl1) if r else None,
                                   _stream(stream)), "svdq_quantize_act")
-    return codes, scales, (xl1 if r else None)
+    return codes, scales, (xl1.view(-1)[:M * r].view(M, r) if r else None)
 
 
 def svdq_pack_lowrank(L1: torch.Tensor, smooth_inv: torch.Tensor | None = None,
@@ -113,6 +121,8 @@ def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int
     """Steps a5..a6: Y [M, N] = Q(X_hat) Q(R)^T + xl1 @ L2 + bias."""
     lib = N.load()
     r = 0 if L2 is None else L2.shape[0]
+    if r and (xl1 is None or xl1.dtype != torch.float32 or xl1.numel() < M * r):
+        raise ValueError("xl1 must be float32 [M, r]")
     f = _fmt(fmt)
     out = N.OUT_F32 if out_dtype == torch.float32 else N.OUT_BF16
     if Y is None:

@@ -23,7 +23,7 @@ EXPORTS = (
     "svdq_status_str", "svdq_version", "svdq_codes_bytes", "svdq_scales_bytes",
     "awq_qweight_bytes", "awq_sz_bytes", "svdq_quantize_act", "svdq_w4a4_linear",
     "awq_w4a16_linear", "svdq_pack", "svdq_unpack", "svdq_check_device_status",
-    "svdq_debug_wait_timeout", "svdq_pack_lowrank",
+    "svdq_debug_wait_timeout", "svdq_pack_lowrank", "svdq_xl1_splits",
 )
 
 _lib = None
@@ -57,6 +57,7 @@ def load() -> ctypes.CDLL:
         "svdq_check_device_status": (_I, [_P]),
         "svdq_debug_wait_timeout": (_I, [_I, _P]),
         "svdq_pack_lowrank": (_I, [_I, _I, _P, _P, _P, _P]),
+        "svdq_xl1_splits": (_I, [_I, _I, _I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

@@ -10,85 +10,104 @@
 // about 2^-17 relative, accumulated in float32 in tensor memory. The quantizer
 // threads therefore only read X and write codes and scales.
 //
-// One CTA owns 128 rows and a contiguous range of 64-column chunks of X. A
-// cluster of `ksplit` CTAs covers all of K for the same 128 rows; their partial
-// sums are added through distributed shared memory in a fixed order.
+// One CTA per SM (a kernel that allocates tensor memory runs one CTA per SM)
+// owns 128 rows and a contiguous range of 64-column chunks of X: the grid
+// splits K into S = svdq_xl1_splits(M, K, r) ranges so that the row blocks times
+// S fill the SMs. Each split writes its own partial down-projection
+// xl1[split][M][r], so no CTA waits for another; a small kernel then adds the S
+// partials in split order into xl1[0].
 //
-// Warp roles (10 warps):
-//   warp 0      TMA producer: X chunk [128 x 64] bf16 (128-byte swizzle), the L1s
-//               hi and lo chunks [r x 64] bf16, and 64 smooth_inv values
+// A ring stage holds two 64-column sub-chunks (when shared memory allows; one
+// for large r). Warp roles (18 warps):
+//   warp 0      TMA producer: per sub-chunk the X tile [128 x 64] bf16 (128-byte
+//               swizzle), the L1s hi and lo tiles [r x 64] bf16, 64 smooth_inv
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
-//   warps 2..9  quantizers; warp q handles rows 16q..16q+15, lane l handles row
-//               16q + l%16 and columns 32(l/16)..32(l/16)+31 of the chunk: two
-//               NVFP4 groups, or half an INT4 group (the other half is lane l^16);
-//               the float32 arithmetic runs on paired (f32x2) instructions
+//   warps 2..17 quantizers; quantizer w takes sub-chunk w / 8 of a stage, rows
+//               16 (w % 8) .. + 15; lane l handles row 16 (w % 8) + l % 16 and
+//               columns 32 (l / 16) .. + 31 of the sub-chunk: two NVFP4 groups, or
+//               half an INT4 group (the other half is lane l ^ 16); the float32
+//               arithmetic runs on paired (f32x2) instructions
 #pragma once
 
 #include "sm100.cuh"
 
 namespace svdq {
 
-constexpr int kQaWarps = 10;
+constexpr int kQaWarps = 18;
 constexpr int kQaThreads = kQaWarps * 32;
-constexpr int kQaQuantWarps = 8;
-constexpr int kQaChunk = 64;                        // columns per stage
+constexpr int kQaQuantWarps = 16;
+constexpr int kQaChunk = 64;                        // columns per sub-chunk
 constexpr int kQaXStageBytes = 128 * kQaChunk * 2;  // 16 KB
 constexpr int kQaSmoothBytes = kQaChunk * 4;        // 256 B
+constexpr int kQaSmTarget = 148;                    // B200 SMs: the K split fills them
+
+// Number of K splits (partial down-projections) for an M x K activation: the
+// largest power of two <= 8 that keeps (row blocks x splits) within the SMs.
+__host__ __device__ inline int qa_splits(int M, int K) {
+  const int row_blocks = (M + 127) / 128;
+  const int kc_total = K / kQaChunk;
+  int s = 1;
+  while (s * 2 <= 8 && s * 2 <= kc_total && row_blocks * s * 2 <= kQaSmTarget) s *= 2;
+  return s;
+}
 
 struct QuantActParams {
   int M, K, r;
-  int ksplit;      // CTAs per cluster along K (1, 2, 4 or 8)
+  int ksplit;      // K ranges (grid.x); split ks writes xl1[ks]
   int stages;      // ring depth
+  int spc;         // sub-chunks per stage (1 or 2)
   int m_pad;       // M rounded up to 128
   const float* smooth_inv;
   uint8_t* codes;
   uint8_t* scales;
-  float* xl1;
+  float* xl1;      // [ksplit][M][r]
   uint32_t* status;
 };
 
 struct QaSmem {
   // byte offsets from the 1024-aligned dynamic shared memory base
-  uint32_t ring, stage_bytes, l1_off, sm_off, table, bars, tmem_slot;
+  uint32_t ring, sub_bytes, stage_bytes, l1_off, sm_off, table, bars, tmem_slot;
 };
 
-__host__ __device__ inline QaSmem qa_smem_layout(int r, int stages) {
+__host__ __device__ inline QaSmem qa_smem_layout(int r, int stages, int spc) {
   QaSmem s;
   s.ring = 0;
   s.l1_off = kQaXStageBytes;                       // hi plane, then lo plane
   s.sm_off = kQaXStageBytes + 2 * r * 128;         // smooth_inv chunk
-  s.stage_bytes = (s.sm_off + kQaSmoothBytes + 1023) / 1024 * 1024;
+  s.sub_bytes = (s.sm_off + kQaSmoothBytes + 1023) / 1024 * 1024;
+  s.stage_bytes = spc * s.sub_bytes;
   s.table = s.ring + stages * s.stage_bytes;       // E4M3 (value, reciprocal) x 128
   s.bars = s.table + 128 * 8;
   s.tmem_slot = s.bars + 8 * (2 * stages + 1);
   return s;
 }
 
-__host__ inline size_t qa_smem_bytes(int r, int stages) {
-  QaSmem s = qa_smem_layout(r, stages);
+__host__ inline size_t qa_smem_bytes(int r, int stages, int spc) {
+  QaSmem s = qa_smem_layout(r, stages, spc);
   return s.tmem_slot + 16 + 1024;  // + alignment slack
 }
 
 template <int kFmt>  // 0: NVFP4 (E2M1, UE4M3 per 16), 1: INT4 (FP16 per 64)
-__global__ void __launch_bounds__(kQaThreads, 3)
+__global__ void __launch_bounds__(kQaThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_l1, const QuantActParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const QaSmem L = qa_smem_layout(p.r, p.stages);
+  const QaSmem L = qa_smem_layout(p.r, p.stages, p.spc);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int NS = p.stages;
   const int r = p.r;
   const bool smoothing = p.smooth_inv != nullptr;
 
-  const int ks = blockIdx.x % p.ksplit;
+  const int ks = blockIdx.x;
   const int rb = blockIdx.y;
   const int kc_total = p.K / kQaChunk;
   const int kc0 = ks * kc_total / p.ksplit;
   const int kc1 = (ks + 1) * kc_total / p.ksplit;
   const int nchunks = kc1 - kc0;
+  const int nstage = (nchunks + p.spc - 1) / p.spc;  // ring uses of this CTA
 
   auto bar_full = [&](int s) { return sbase + L.bars + 8 * s; };
   auto bar_empty = [&](int s) { return sbase + L.bars + 8 * (NS + s); };
@@ -127,40 +146,46 @@ __global__ void __launch_bounds__(kQaThreads, 3)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (elect_one()) {
-      const uint32_t tx = kQaXStageBytes + 2 * r * 128 + (smoothing ? kQaSmoothBytes : 0);
-      for (int i = 0; i < nchunks; ++i) {
+      const uint32_t sub_tx = kQaXStageBytes + 2 * r * 128 + (smoothing ? kQaSmoothBytes : 0);
+      for (int i = 0; i < nstage; ++i) {
         const int s = i % NS;
         if (!mbar_wait(bar_empty(s), ((i / NS) & 1) ^ 1, p.status)) break;
-        const int kc = kc0 + i;
-        mbar_arrive_expect_tx(bar_full(s), tx);
-        tma_load_2d(x_stage(s), &tm_x, bar_full(s), kc * kQaChunk, rb * 128);
-        if (r > 0) {
-          tma_load_2d(x_stage(s) + L.l1_off, &tm_l1, bar_full(s), kc * kQaChunk, 0);
-          tma_load_2d(x_stage(s) + L.l1_off + r * 128, &tm_l1, bar_full(s), kc * kQaChunk, r);
+        const int nsub = min(p.spc, nchunks - i * p.spc);
+        mbar_arrive_expect_tx(bar_full(s), nsub * sub_tx);
+        for (int u = 0; u < nsub; ++u) {
+          const int kc = kc0 + i * p.spc + u;
+          const uint32_t base = x_stage(s) + u * L.sub_bytes;
+          tma_load_2d(base, &tm_x, bar_full(s), kc * kQaChunk, rb * 128);
+          if (r > 0) {
+            tma_load_2d(base + L.l1_off, &tm_l1, bar_full(s), kc * kQaChunk, 0);
+            tma_load_2d(base + L.l1_off + r * 128, &tm_l1, bar_full(s), kc * kQaChunk, r);
+          }
+          if (smoothing)
+            bulk_load(base + L.sm_off, p.smooth_inv + kc * kQaChunk, kQaSmoothBytes, bar_full(s));
         }
-        if (smoothing)
-          bulk_load(x_stage(s) + L.sm_off, p.smooth_inv + kc * kQaChunk, kQaSmoothBytes,
-                    bar_full(s));
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (r > 0 && elect_one()) {
       const uint32_t idesc = idesc_bf16_f32(128, r, false, false);
-      for (int i = 0; i < nchunks; ++i) {
+      for (int i = 0; i < nstage; ++i) {
         const int s = i % NS;
         if (!mbar_wait(bar_full(s), (i / NS) & 1, p.status)) break;
         tc_fence_after();
+        const int nsub = min(p.spc, nchunks - i * p.spc);
+        for (int u = 0; u < nsub; ++u) {
+          const uint32_t base = x_stage(s) + u * L.sub_bytes;
 #pragma unroll
-        for (int kk = 0; kk < kQaChunk / 16; ++kk) {
-          // A: the X tile, 128 rows x 128 B, 128-byte swizzle; 16 K = 32 B
-          const uint64_t ad = smem_desc(x_stage(s) + kk * 32, 16, 1024, kSwizzle128B);
-          // B: L1s hi / lo planes, r rows x 128 B each, 128-byte swizzle
-          const uint64_t bh = smem_desc(x_stage(s) + L.l1_off + kk * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bl =
-              smem_desc(x_stage(s) + L.l1_off + r * 128 + kk * 32, 16, 1024, kSwizzle128B);
-          mma_f16(tmem_base, ad, bh, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_f16(tmem_base, ad, bl, idesc, 1u);
+          for (int kk = 0; kk < kQaChunk / 16; ++kk) {
+            // A: the X tile, 128 rows x 128 B, 128-byte swizzle; 16 K = 32 B
+            const uint64_t ad = smem_desc(base + kk * 32, 16, 1024, kSwizzle128B);
+            // B: L1s hi / lo planes, r rows x 128 B each, 128-byte swizzle
+            const uint64_t bh = smem_desc(base + L.l1_off + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bl = smem_desc(base + L.l1_off + r * 128 + kk * 32, 16, 1024, kSwizzle128B);
+            mma_f16(tmem_base, ad, bh, idesc, (i > 0 || u > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(tmem_base, ad, bl, idesc, 1u);
+          }
         }
         tc_commit(bar_empty(s));
       }
@@ -169,173 +194,149 @@ __global__ void __launch_bounds__(kQaThreads, 3)
   } else {
     // ---------------------------------------------------------------- quantizers
     const int qw = warp - 2;
-    const int row = qw * 16 + (lane & 15);
-    const int half = lane >> 4;  // which 32 columns of the chunk
+    const int sub = p.spc == 2 ? qw >> 3 : 0;     // which sub-chunk of a stage
+    const bool active = p.spc == 2 || qw < 8;    // one sub-chunk per stage: warps 0..7 quantize
+    const int row = (qw & 7) * 16 + (lane & 15);
+    const int half = lane >> 4;  // which 32 columns of the sub-chunk
     const int m = rb * 128 + row;
     const bool row_ok = m < p.M;
     bool ok = true;
-    for (int i = 0; i < nchunks; ++i) {
+    for (int i = 0; i < nstage; ++i) {
       const int s = i % NS;
-      const int kc = kc0 + i;
       ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status);
       if (!ok) break;
-      // -- 32 bf16 of this row from the 128B-swizzled X tile, as float32 pairs
-      uint64_t xp[16];
-      {
-        const uint32_t rowbase = x_stage(s) + row * 128;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int c = 4 * half + h;
-          uint32_t v0, v1, v2, v3;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
-                       : "r"(rowbase + ((c ^ (row & 7)) << 4)));
-          const uint32_t w[4] = {v0, v1, v2, v3};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            xp[4 * h + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+      const int kc = kc0 + i * p.spc + sub;
+      if (!active || kc >= kc1) {
+        // nothing of this stage for this warp
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+        continue;
+      }
+      const uint32_t sub_base = x_stage(s) + sub * L.sub_bytes;
+        // -- 32 bf16 of this row from the 128B-swizzled X tile, as float32 pairs
+        uint64_t xp[16];
+        {
+          const uint32_t rowbase = sub_base + row * 128;
+  #pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int c = 4 * half + h;
+            uint32_t v0, v1, v2, v3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                         : "r"(rowbase + ((c ^ (row & 7)) << 4)));
+            const uint32_t w[4] = {v0, v1, v2, v3};
+  #pragma unroll
+            for (int j = 0; j < 4; ++j)
+              xp[4 * h + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+          }
         }
-      }
-      // -- a1: smoothing, one float32 multiply per element
-      if (smoothing) {
-        const float4* sp = reinterpret_cast<const float4*>(smem + (x_stage(s) - sbase) + L.sm_off) +
-                           8 * half;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 sv = sp[j];
-          xp[2 * j] = f2_mul(xp[2 * j], f2_pack(sv.x, sv.y));
-          xp[2 * j + 1] = f2_mul(xp[2 * j + 1], f2_pack(sv.z, sv.w));
+        // -- a1: smoothing, one float32 multiply per element
+        if (smoothing) {
+          const float4* sp = reinterpret_cast<const float4*>(smem + (sub_base - sbase) + L.sm_off) +
+                             8 * half;
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 sv = sp[j];
+            xp[2 * j] = f2_mul(xp[2 * j], f2_pack(sv.x, sv.y));
+            xp[2 * j + 1] = f2_mul(xp[2 * j + 1], f2_pack(sv.z, sv.w));
+          }
         }
-      }
-      // this warp no longer reads the stage's shared memory
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty(s));
-      // -- a2 + a3: group scale and codes
-      float xh[32];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float2 v = f2_unpack(xp[j]);
-        xh[2 * j] = v.x;
-        xh[2 * j + 1] = v.y;
-      }
-      uint32_t code[4];
-      if (kFmt == 0) {
-        uint32_t sc[2];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
+        // this warp no longer reads the stage's shared memory
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+        // -- a2 + a3: group scale and codes
+        float xh[32];
+  #pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 v = f2_unpack(xp[j]);
+          xh[2 * j] = v.x;
+          xh[2 * j + 1] = v.y;
+        }
+        uint32_t code[4];
+        if (kFmt == 0) {
+          uint32_t sc[2];
+  #pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            float amax = 0.0f;
+  #pragma unroll
+            for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[16 * g + j]));
+            sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
+            const float2 vr = table[sc[g]];  // (decoded scale, its reciprocal)
+            const uint64_t rcp2 = f2_pack(vr.y, vr.y);
+            float y0[8], y1[8];
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 a = f2_unpack(f2_mul(xp[8 * g + j], rcp2));
+              const float2 b = f2_unpack(f2_mul(xp[8 * g + 4 + j], rcp2));
+              y0[2 * j] = a.x;
+              y0[2 * j + 1] = a.y;
+              y1[2 * j] = b.x;
+              y1[2 * j + 1] = b.y;
+            }
+            const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
+            code[2 * g] = live ? e2m1x8(y0) : 0u;
+            code[2 * g + 1] = live ? e2m1x8(y1) : 0u;
+          }
+          // the row's four scale bytes: groups 2 half, 2 half + 1 here, the others in lane ^ 16
+          const uint32_t mine = sc[0] | (sc[1] << 8);
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
+          if (half == 0) {
+            const uint32_t word = mine | (other << 16);
+            const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
+            *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
+                word;
+          }
+        } else {
           float amax = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[16 * g + j]));
-          sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
-          const float2 vr = table[sc[g]];  // (decoded scale, its reciprocal)
-          const uint64_t rcp2 = f2_pack(vr.y, vr.y);
-          float y0[8], y1[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 a = f2_unpack(f2_mul(xp[8 * g + j], rcp2));
-            const float2 b = f2_unpack(f2_mul(xp[8 * g + 4 + j], rcp2));
-            y0[2 * j] = a.x;
-            y0[2 * j + 1] = a.y;
-            y1[2 * j] = b.x;
-            y1[2 * j + 1] = b.y;
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xh[j]));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+          const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
+          const float sval = __half2float(hs);
+  #pragma unroll
+          for (int w = 0; w < 4; ++w) code[w] = 0u;
+          if (sval != 0.0f) {
+            const float rcp = __frcp_rn(sval);
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              int v = __float2int_rn(__fmul_rn(xh[j], rcp));
+              v = max(-7, min(7, v));
+              // tiled INT4 codes are sign-magnitude nibbles
+              const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
+              code[j >> 3] |= nib << (4 * (j & 7));
+            }
           }
-          const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
-          code[2 * g] = live ? e2m1x8(y0) : 0u;
-          code[2 * g + 1] = live ? e2m1x8(y1) : 0u;
+          if (half == 0)
+            reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] =
+                hs;
         }
-        // the row's four scale bytes: groups 2 half, 2 half + 1 here, the others in lane ^ 16
-        const uint32_t mine = sc[0] | (sc[1] << 8);
-        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
-        if (half == 0) {
-          const uint32_t word = mine | (other << 16);
-          const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
-          *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
-              word;
+        if (row_ok) {
+          *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + half * 16) =
+              make_uint4(code[0], code[1], code[2], code[3]);
         }
-      } else {
-        float amax = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xh[j]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-        const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
-        const float sval = __half2float(hs);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) code[w] = 0u;
-        if (sval != 0.0f) {
-          const float rcp = __frcp_rn(sval);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            int v = __float2int_rn(__fmul_rn(xh[j], rcp));
-            v = max(-7, min(7, v));
-            // tiled INT4 codes are sign-magnitude nibbles
-            const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
-            code[j >> 3] |= nib << (4 * (j & 7));
-          }
-        }
-        if (half == 0)
-          reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] =
-              hs;
-      }
-      if (row_ok) {
-        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + half * 16) =
-            make_uint4(code[0], code[1], code[2], code[3]);
-      }
     }
     // ------------------------------------------------------------ xl1 epilogue
-    // The reduction buffer reuses the ring: every quantizer warp must be done
-    // reading X before any of them writes partial sums there.
-    if (r > 0 && p.ksplit > 1) asm volatile("bar.sync 1, %0;" ::"n"(kQaQuantWarps * 32) : "memory");
+    // this split's partial down-projection of the CTA's 128 rows
     if (r > 0 && ok && mbar_wait(bar_acc, 0, p.status)) {
       tc_fence_after();
       const int quad = warp & 3;         // tensor-memory lanes this warp may read
-      const int part = (warp - 2) >> 2;  // which half of the r columns
+      const int part = (warp - 2) >> 2;  // which quarter of the r columns
       const int trow = quad * 32 + lane;
-      const int ncol = r / 2, c_begin = part * ncol;
-      const int rs = r + 4;  // padded row stride (floats) of the reduction buffer
-      float* red = reinterpret_cast<float*>(smem + L.ring);
+      const int ncol = r / 4, c_begin = part * ncol;
       const int tm = rb * 128 + trow;
+      float* dst = p.xl1 + (static_cast<size_t>(ks) * p.M + tm) * r;
       for (int c = c_begin; c < c_begin + ncol; c += 4) {
         uint32_t v[4];
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
                      : "r"(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c));
         tmem_ld_wait();
-        const float4 f = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]),
-                                     __uint_as_float(v[2]), __uint_as_float(v[3]));
-        if (p.ksplit == 1) {
-          if (tm < p.M) *reinterpret_cast<float4*>(p.xl1 + static_cast<size_t>(tm) * r + c) = f;
-        } else {
-          *reinterpret_cast<float4*>(red + trow * rs + c) = f;
-        }
+        if (tm < p.M)
+          *reinterpret_cast<float4*>(dst + c) =
+              make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                          __uint_as_float(v[3]));
       }
     }
-  }
-
-  // ---------------------------------------------------------- cluster reduction
-  if (r > 0 && p.ksplit > 1) {
-    cluster_sync();  // every CTA's partial sums are in its shared memory
-    if (warp >= 2) {
-      const int rows_per = 128 / p.ksplit;
-      const int units = rows_per * (r / 4);
-      const int rs = r + 4;
-      const uint32_t red = sbase + L.ring;
-      for (int u = threadIdx.x - 64; u < units; u += kQaQuantWarps * 32) {
-        const int trow = ks * rows_per + u / (r / 4);
-        const int c = (u % (r / 4)) * 4;
-        const uint32_t off = red + (trow * rs + c) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int pr = 0; pr < p.ksplit; ++pr) {
-          const float4 v = ld_dsmem_f4(map_peer_smem(off, pr));
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-        }
-        const int tm = rb * 128 + trow;
-        if (tm < p.M) *reinterpret_cast<float4*>(p.xl1 + static_cast<size_t>(tm) * r + c) = acc;
-      }
-    }
-    cluster_sync();  // keep shared memory alive until every peer has read it
   }
 
   tc_fence_before();
@@ -343,6 +344,23 @@ __global__ void __launch_bounds__(kQaThreads, 3)
   if (warp == 1 && r > 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// The K splits' partial down-projections, added in split order into split 0:
+// xl1[0] = ((xl1[0] + xl1[1]) + ...) + xl1[S-1]; n4 float4 per split.
+__global__ void xl1_reduce_kernel(float4* xl1, int splits, size_t n4) {
+  for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n4;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float4 v = xl1[t];
+    for (int sp = 1; sp < splits; ++sp) {
+      const float4 u = xl1[sp * n4 + t];
+      v.x += u.x;
+      v.y += u.y;
+      v.z += u.z;
+      v.w += u.w;
+    }
+    xl1[t] = v;
   }
 }
 

@@ -250,6 +250,11 @@ size_t awq_sz_bytes(int N, int K) {
   return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 64) * 4;
 }
 
+int svdq_xl1_splits(int M, int K, int r) {
+  if (M < 1 || K < 64 || K % 64 || !rank_ok(r)) return 0;
+  return r == 0 ? 1 : qa_splits(M, K);
+}
+
 svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
                               const float* smooth_inv, const void* L1s, void* codes,
                               void* scales, float* xl1, svdq_stream_t stream) {
@@ -277,45 +282,26 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   }
 
   const int row_blocks = (M + 127) / 128;
-  const int kc_total = K / 64;
-  // Ring depth: two CTAs per SM when at least 3 stages fit in half the shared
-  // memory, else one CTA per SM with up to 8 stages.
-  const QaSmem lay = qa_smem_layout(r, 1);
-  const int stage_bytes = static_cast<int>(lay.stage_bytes);
-  const int fixed = static_cast<int>(qa_smem_bytes(r, 0));
-  const int red_bytes = r > 0 ? 128 * (r + 4) * 4 : 0;  // reduction buffer, reuses the ring
-  auto fits = [&](int st, int budget) {
-    return st >= 2 && fixed + st * stage_bytes <= budget && red_bytes <= st * stage_bytes;
-  };
-  // Two configurations: two CTAs per SM (ring in half the shared memory, at
-  // least 3 stages) or one CTA per SM (up to 8 stages). Two per SM is used only
-  // when the grid has more CTAs than SMs: the block scheduler fills SMs two at a
-  // time, so a smaller grid would leave SMs idle.
-  int stages2 = 0, stages1 = 0;
-  const int half_budget = 113 * 1024, full_budget = 227 * 1024;
-  for (int st = 8; st >= 3 && stages2 == 0; --st)
-    if (fits(st, half_budget)) stages2 = st;
-  for (int st = 8; st >= 2 && stages1 == 0; --st)
-    if (fits(st, full_budget)) stages1 = st;
-  if (stages1 == 0) return SVDQ_ERR_UNSUPPORTED;
-  // K split: the largest power of two (<= 8, <= K/64) whose CTAs fit in one wave
-  const int max_ctas = (stages2 ? 2 : 1) * d->num_sms;
-  int ksplit = 1;
-  while (ksplit * 2 <= 8 && ksplit * 2 <= kc_total && row_blocks * ksplit * 2 <= max_ctas)
-    ksplit *= 2;
-  const bool two_per_sm = stages2 != 0 && row_blocks * ksplit > d->num_sms;
-  const int stages = two_per_sm ? stages2 : stages1;
-  const int per_sm = two_per_sm ? 2 : 1;
-  const size_t smem_bytes = qa_smem_bytes(r, stages);
+  // One CTA per SM (the kernel allocates tensor memory), K split into
+  // qa_splits(M, K) ranges; ring stages of two 64-column sub-chunks where at
+  // least two such stages fit, else of one.
+  const int ksplit = qa_splits(M, K);
+  const size_t budget = 227 * 1024;
+  int spc = 0, stages = 0;
+  for (int c = 2; c >= 1 && stages == 0; --c)
+    for (int st = 8; st >= 2 && stages == 0; --st)
+      if (qa_smem_bytes(r, st, c) <= budget) {
+        spc = c;
+        stages = st;
+      }
+  if (stages == 0) return SVDQ_ERR_UNSUPPORTED;
+  const size_t smem_bytes = qa_smem_bytes(r, stages, spc);
   auto kern = format == SVDQ_NVFP4_G16 ? quantize_act_kernel<0> : quantize_act_kernel<1>;
-  if (debug_on()) {
-    int occ = -1;
-    (void)cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kQaThreads, smem_bytes);
+  if (debug_on())
     std::fprintf(stderr,
-                 "svdq_quantize_act: M=%d K=%d r=%d stages=%d per_sm=%d ksplit=%d grid=%d smem=%zu "
-                 "occupancy=%d\n",
-                 M, K, r, stages, per_sm, ksplit, ksplit * row_blocks, smem_bytes, occ);
-  }
+                 "svdq_quantize_act: M=%d K=%d r=%d stages=%d x %d sub-chunks ksplit=%d grid=%d "
+                 "smem=%zu\n",
+                 M, K, r, stages, spc, ksplit, ksplit * row_blocks, smem_bytes);
 
   QuantActParams p;
   p.M = M;
@@ -323,31 +309,22 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   p.r = r;
   p.ksplit = ksplit;
   p.stages = stages;
+  p.spc = spc;
   p.m_pad = static_cast<int>(pad128(M));
   p.smooth_inv = smooth_inv;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
   p.xl1 = xl1;
   p.status = d->status;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ksplit, row_blocks, 1);
-  cfg.blockDim = dim3(kQaThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = ksplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = (r > 0 && ksplit > 1) ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tm_x, tm_l1, p);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return SVDQ_ERR_CUDA;
+  kern<<<dim3(ksplit, row_blocks, 1), kQaThreads, smem_bytes, static_cast<cudaStream_t>(stream)>>>(
+      tm_x, tm_l1, p);
+  if (r > 0 && ksplit > 1) {
+    // xl1[0] += xl1[1] + ... + xl1[S-1], in order
+    const size_t n4 = static_cast<size_t>(M) * r / 4;
+    xl1_reduce_kernel<<<grid_for(n4, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<float4*>(xl1), ksplit, n4);
   }
-  return SVDQ_OK;
+  return launch_status();
 }
 
 svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,

@@ -7,7 +7,8 @@ from __future__ import annotations
 
 import torch
 
-from . import awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_scales_bytes, svdq_w4a4_linear
+from . import (awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_scales_bytes,
+               svdq_w4a4_linear, svdq_xl1_splits)
 
 
 class SvdqW4A4Linear:
@@ -24,13 +25,15 @@ class SvdqW4A4Linear:
                                  device=dev)
         self.scales = torch.empty(svdq_scales_bytes(self.fmt, max_tokens, self.K), dtype=torch.uint8,
                                   device=dev)
-        self.xl1 = torch.empty((max_tokens, self.r), dtype=torch.float32, device=dev) if self.r else None
+        # the down-projection's partial sums: at most 8 splits of max_tokens rows
+        self.xl1 = (torch.empty(8 * max_tokens * self.r, dtype=torch.float32, device=dev)
+                    if self.r else None)
 
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         M = x.shape[0]
         if M > self.max_tokens:
             raise ValueError(f"{M} tokens > workspace for {self.max_tokens}")
-        xl1 = self.xl1[:M] if self.r else None
+        xl1 = self.xl1[:svdq_xl1_splits(M, self.K, self.r) * M * self.r] if self.r else None
         codes, scales, xl1 = svdq_quantize_act(x, self.w["L1s"], self.w["smooth_inv"], fmt=self.fmt,
                                                codes=self.codes, scales=self.scales, xl1=xl1,
                                                stream=stream)

@@ -89,6 +89,15 @@ size_t awq_qweight_bytes(int N, int K);
 size_t awq_sz_bytes(int N, int K);
 
 /*
+ * svdq_xl1_splits -- S, the number of [M, r] slices of the xl1 buffer that
+ * svdq_quantize_act needs for an M x K activation with rank r (it splits K into
+ * S ranges): the largest power of two <= 8 (and <= K/64) that keeps
+ * ceil(M/128) * S within the 148 SMs of a B200; 1 when r == 0. A pure function
+ * of its arguments; 0 for an invalid request.
+ */
+int svdq_xl1_splits(int M, int K, int r);
+
+/*
  * svdq_quantize_act -- steps a1..a4: smooth, group-scale, quantize + pack the
  * activations, and the rank-r down-projection of the smoothed activations, in
  * one pass over X (Nunchaku README, "Engine design" (b): the down projection and
@@ -107,10 +116,14 @@ size_t awq_sz_bytes(int N, int K);
  *            NULL iff r == 0
  * codes      device, svdq_codes_bytes(format, M, K) bytes, written (tiled form)
  * scales     device, svdq_scales_bytes(format, M, K) bytes, written (padding rows too)
- * xl1        device, float32 [M, r], written; NULL iff r == 0
+ * xl1        device, float32 [S][M][r] with S = svdq_xl1_splits(M, K, r): on
+ *            return its first [M, r] slice holds x_hat L1; the other S - 1
+ *            slices are the call's working space (the down-projections of S
+ *            ranges of K, added in order into the first); NULL iff r == 0
  * Codes and scales are bit-exact functions of the inputs. xl1 is computed on the
  * tensor cores as X (hi + lo) with float32 accumulation, which equals x_hat L1 to
- * about 2^-17 relative per term. This call also serves as the weight quantizer
+ * about 2^-17 relative per term. The K ranges let every SM work on the pass
+ * without any CTA waiting for another. This call also serves as the weight quantizer
  * (residual R given as bf16, smooth_inv NULL, r 0).
  */
 svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
@@ -127,7 +140,8 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
  *          + sum_j xl1[m,j] L2[j,n] + bias[n]
  *
  * a_codes, a_scales  device, activation codes/scales from svdq_quantize_act (M rows)
- * xl1                device, float32 [M, r]; NULL iff r == 0
+ * xl1                device, float32 [M, r] (the first slice of svdq_quantize_act's
+ *                    xl1); NULL iff r == 0
  * w_codes, w_scales  device, weight codes/scales in the same formats (N rows)
  * L2                 device, bf16 [r, N]; NULL iff r == 0
  * bias               device, bf16 [N], or NULL

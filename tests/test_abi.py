@@ -77,3 +77,14 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.svdq_pack(0, 0, 10, 64, good, good, good, good, good, None) == 1  # zeros for ACT
     assert lib.svdq_pack(2, 0, 10, 64, good, good, None, good, good, None) == 1  # no zeros for AWQ
     assert lib.svdq_debug_wait_timeout(0, None) == 1
+
+
+def test_xl1_splits_is_a_pure_function_of_the_shape(lib):
+    # ceil(M/128) row blocks times S stays within 148 SMs; S a power of two <= 8, <= K/64
+    assert lib.svdq_xl1_splits(4608, 3072, 32) == 4      # 36 row blocks -> 144 CTAs
+    assert lib.svdq_xl1_splits(18432, 3072, 32) == 1     # 144 row blocks
+    assert lib.svdq_xl1_splits(256, 512, 16) == 8        # 2 row blocks, K/64 = 8
+    assert lib.svdq_xl1_splits(256, 128, 16) == 2        # K/64 = 2 caps it
+    assert lib.svdq_xl1_splits(4608, 3072, 0) == 1       # no low-rank branch
+    assert lib.svdq_xl1_splits(4608, 3000, 32) == 0      # K not a multiple of 64
+    assert lib.svdq_xl1_splits(4608, 3072, 24) == 0      # rank not a multiple of 16

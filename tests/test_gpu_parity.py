@@ -60,7 +60,8 @@ def _quantize_gpu(bq, layer, X_bits, fmt, with_lowrank=True, smooth=True):
     L1s = C.bf16_tensor(F.bf16_bits(LO.lowrank_operand(layer["L1"], layer["smooth_inv"] if smooth else None))) if r else None
     codes, scales, xl1 = bq.svdq_quantize_act(X, L1s, si, fmt=fmt)
     assert bq.svdq_check_device_status() == 0
-    return codes.cpu().numpy(), scales.cpu().numpy(), (xl1.cpu().numpy() if xl1 is not None else None)
+    return codes.cpu().numpy(), scales.cpu().numpy(), (
+        xl1.cpu().numpy().astype(np.float64) if xl1 is not None else None)
 
 
 @pytest.mark.parametrize("shape", SMALL + SMALL_INT4[:2], ids=lambda s: s.name)
@@ -78,7 +79,7 @@ def test_quantize_act_matches_oracle(bq, shape):
     assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:5]}"
     if shape.r:
         ref = S.down_proj(xhat, layer["L1"])
-        err = np.abs(xl1.astype(np.float64) - ref)
+        err = np.abs(xl1 - ref)
         assert np.all(err <= C.xl1_bound(xhat, layer["L1"])), f"xl1 max err {err.max():.3e}"
 
 
