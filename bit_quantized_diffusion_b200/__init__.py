@@ -99,6 +99,39 @@ def svdq_quantize_act(X: torch.Tensor, L1s: torch.Tensor | None = None,
     return codes, scales, (xl1.view(-1)[:M * r].view(M, r) if r else None)
 
 
+def svdq_quantize_act_noalloc(X: torch.Tensor, L1s: torch.Tensor | None = None,
+                              smooth_inv: torch.Tensor | None = None, fmt="nvfp4",
+                              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                              xl1: torch.Tensor | None = None, stream=None):
+    """svdq_quantize_act with xl1 only [M, r]: the library's static device array
+    holds the K splits' partial sums (see include/svdq.h for the limit)."""
+    lib = N.load()
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    r = 0 if L1s is None else L1s.shape[1]
+    f = _fmt(fmt)
+    dev = X.device
+    if codes is None:
+        codes = torch.empty(lib.svdq_codes_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(lib.svdq_scales_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    if r and xl1 is None:
+        xl1 = torch.empty((M, r), dtype=torch.float32, device=dev)
+    _need(codes, lib.svdq_codes_bytes(f, M, K), "codes")
+    _need(scales, lib.svdq_scales_bytes(f, M, K), "scales")
+    if L1s is not None and (L1s.dtype != torch.bfloat16 or tuple(L1s.shape) != (2, r, K)):
+        raise ValueError("L1s must be bf16 [2, r, K]")
+    if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
+        raise ValueError("smooth_inv must be float32 [K]")
+    if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < M * r):
+        raise ValueError("xl1 must be float32 [M, r]")
+    N.check(lib.svdq_quantize_act_noalloc(f, M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(L1s),
+                                          _ptr(codes), _ptr(scales), _ptr(xl1) if r else None,
+                                          _stream(stream)), "svdq_quantize_act_noalloc")
+    return codes, scales, (xl1.view(-1)[:M * r].view(M, r) if r else None)
+
+
 def svdq_pack_lowrank(L1: torch.Tensor, smooth_inv: torch.Tensor | None = None,
                       L1s: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """L1 [K, r] bf16 (+ smooth_inv [K] f32) -> the [2, r, K] bf16 down-projection operand."""

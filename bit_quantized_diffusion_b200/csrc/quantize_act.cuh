@@ -13,9 +13,9 @@
 // One CTA per SM (a kernel that allocates tensor memory runs one CTA per SM)
 // owns 128 rows and a contiguous range of 64-column chunks of X: the grid
 // splits K into S = svdq_xl1_splits(M, K, r) ranges so that the row blocks times
-// S fill the SMs. Each split writes its own partial down-projection
-// xl1[split][M][r], so no CTA waits for another; a small kernel then adds the S
-// partials in split order into xl1[0].
+// S fill the SMs. Each split writes its own partial down-projection (split 0
+// into xl1, the others into working space), so no CTA waits for another; a
+// small kernel then adds the S partials in split order into xl1.
 //
 // A ring stage holds two 64-column sub-chunks (when shared memory allows; one
 // for large r). Warp roles (18 warps):
@@ -60,7 +60,8 @@ struct QuantActParams {
   const float* smooth_inv;
   uint8_t* codes;
   uint8_t* scales;
-  float* xl1;      // [ksplit][M][r]
+  float* xl1;      // split 0 (and, after the reduction, the sum): [M][r]
+  float* xl1_rest; // splits 1 .. ksplit - 1: [ksplit - 1][M][r]
   uint32_t* status;
 };
 
@@ -324,7 +325,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       const int trow = quad * 32 + lane;
       const int ncol = r / 4, c_begin = part * ncol;
       const int tm = rb * 128 + trow;
-      float* dst = p.xl1 + (static_cast<size_t>(ks) * p.M + tm) * r;
+      float* dst = (ks == 0 ? p.xl1 : p.xl1_rest + static_cast<size_t>(ks - 1) * p.M * r) +
+                   static_cast<size_t>(tm) * r;
       for (int c = c_begin; c < c_begin + ncol; c += 4) {
         uint32_t v[4];
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
@@ -348,13 +350,13 @@ __global__ void __launch_bounds__(kQaThreads, 1)
 }
 
 // The K splits' partial down-projections, added in split order into split 0:
-// xl1[0] = ((xl1[0] + xl1[1]) + ...) + xl1[S-1]; n4 float4 per split.
-__global__ void xl1_reduce_kernel(float4* xl1, int splits, size_t n4) {
+// xl1 = ((xl1 + rest[0]) + ...) + rest[S-2]; n4 float4 per split.
+__global__ void xl1_reduce_kernel(float4* xl1, const float4* rest, int splits, size_t n4) {
   for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n4;
        t += static_cast<size_t>(gridDim.x) * blockDim.x) {
     float4 v = xl1[t];
     for (int sp = 1; sp < splits; ++sp) {
-      const float4 u = xl1[sp * n4 + t];
+      const float4 u = rest[(sp - 1) * n4 + t];
       v.x += u.x;
       v.y += u.y;
       v.z += u.z;

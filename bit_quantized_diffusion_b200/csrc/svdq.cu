@@ -23,6 +23,13 @@ using namespace svdq;
 
 __device__ uint32_t g_svdq_status;
 
+// Working space of svdq_quantize_act_noalloc: the partial down-projections of
+// K splits 1 .. S-1, (S - 1) * M * r floats at most kXl1ScratchFloats (8 MiB).
+// Nothing in it needs to start at zero (each call writes every element it
+// reads); two such calls in flight at the same time race on it.
+constexpr size_t kXl1ScratchFloats = size_t(1) << 21;
+static __device__ __align__(256) float g_xl1_scratch[kXl1ScratchFloats];
+
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
@@ -31,6 +38,7 @@ struct DeviceInfo {
   int gemm_pairs = 0;  // co-resident clusters of the CTA-pair GEMM
   int gemm_pair_mode = -1;  // -1: by shape; SVDQ_GEMM_PAIR=0/1 forces single-CTA / CTA-pair tiles
   uint32_t* status = nullptr;
+  float* xl1_scratch = nullptr;  // device address of g_xl1_scratch
 };
 
 std::mutex g_mu;
@@ -61,6 +69,8 @@ svdq_status device_setup(DeviceInfo** out) {
     }
     void* st = nullptr;
     if (cudaGetSymbolAddress(&st, g_svdq_status) != cudaSuccess) return SVDQ_ERR_CUDA;
+    void* scratch = nullptr;  // this device's copy (the device is current here)
+    if (cudaGetSymbolAddress(&scratch, g_xl1_scratch) != cudaSuccess) return SVDQ_ERR_CUDA;
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     const int max_smem = 232448;
@@ -123,6 +133,7 @@ svdq_status device_setup(DeviceInfo** out) {
     }
     if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) d.gemm_pair_mode = std::atoi(e) != 0;
     d.status = static_cast<uint32_t*>(st);
+    d.xl1_scratch = static_cast<float*>(scratch);
     d.ready = true;
   }
   *out = &d;
@@ -210,54 +221,9 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
   return launch_status();
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* svdq_status_str(svdq_status s) {
-  switch (s) {
-    case SVDQ_OK: return "ok";
-    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
-    case SVDQ_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
-    case SVDQ_ERR_UNSUPPORTED: return "unsupported by this build";
-    case SVDQ_ERR_CUDA: return "CUDA error";
-    case SVDQ_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
-  }
-  return "unknown status";
-}
-
-int svdq_version(void) { return 100; }
-
-size_t svdq_codes_bytes(svdq_format f, int rows, int K) {
-  if ((f != SVDQ_NVFP4_G16 && f != SVDQ_INT4_G64) || rows < 1 || K < 64 || K % 64) return 0;
-  return static_cast<size_t>(rows) * (K / 2);
-}
-
-size_t svdq_scales_bytes(svdq_format f, int rows, int K) {
-  if (rows < 1 || K < 64 || K % 64) return 0;
-  if (f == SVDQ_NVFP4_G16) return pad128(rows) * (K / 16);
-  if (f == SVDQ_INT4_G64) return pad128(rows) * (K / 64) * 2;
-  return 0;
-}
-
-size_t awq_qweight_bytes(int N, int K) {
-  if (N < 1 || K < 64 || K % 64) return 0;
-  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 2);
-}
-
-size_t awq_sz_bytes(int N, int K) {
-  if (N < 1 || K < 64 || K % 64) return 0;
-  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 64) * 4;
-}
-
-int svdq_xl1_splits(int M, int K, int r) {
-  if (M < 1 || K < 64 || K % 64 || !rank_ok(r)) return 0;
-  return r == 0 ? 1 : qa_splits(M, K);
-}
-
-svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
-                              const float* smooth_inv, const void* L1s, void* codes,
-                              void* scales, float* xl1, svdq_stream_t stream) {
+svdq_status quantize_act_impl(svdq_format format, int M, int K, int r, const void* X, int ldx,
+                              const float* smooth_inv, const void* L1s, void* codes, void* scales,
+                              float* xl1, bool static_rest, svdq_stream_t stream) {
   if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || K < 64 || K % 64 || !rank_ok(r) || ldx < K) return SVDQ_ERR_INVALID_ARG;
   if (X == nullptr || codes == nullptr || scales == nullptr) return SVDQ_ERR_INVALID_ARG;
@@ -314,7 +280,19 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
   p.smooth_inv = smooth_inv;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
+  // splits 1 .. S-1: the rest of the caller's buffer, or the library's static
+  // working space (svdq_quantize_act_noalloc)
+  const size_t rest_floats = static_cast<size_t>(ksplit - 1) * M * r;
+  if (static_rest && r > 0 && rest_floats > kXl1ScratchFloats) {
+    if (debug_on())
+      std::fprintf(stderr,
+                   "svdq_quantize_act_noalloc: needs %zu floats of working space, the static "
+                   "array holds %zu\n",
+                   rest_floats, kXl1ScratchFloats);
+    return SVDQ_ERR_UNSUPPORTED;
+  }
   p.xl1 = xl1;
+  p.xl1_rest = r > 0 ? (static_rest ? d->xl1_scratch : xl1 + static_cast<size_t>(M) * r) : nullptr;
   p.status = d->status;
   kern<<<dim3(ksplit, row_blocks, 1), kQaThreads, smem_bytes, static_cast<cudaStream_t>(stream)>>>(
       tm_x, tm_l1, p);
@@ -322,9 +300,69 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
     // xl1[0] += xl1[1] + ... + xl1[S-1], in order
     const size_t n4 = static_cast<size_t>(M) * r / 4;
     xl1_reduce_kernel<<<grid_for(n4, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<float4*>(xl1), ksplit, n4);
+        reinterpret_cast<float4*>(xl1), reinterpret_cast<const float4*>(p.xl1_rest), ksplit, n4);
   }
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svdq_status_str(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported by this build";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+  }
+  return "unknown status";
+}
+
+int svdq_version(void) { return 100; }
+
+size_t svdq_codes_bytes(svdq_format f, int rows, int K) {
+  if ((f != SVDQ_NVFP4_G16 && f != SVDQ_INT4_G64) || rows < 1 || K < 64 || K % 64) return 0;
+  return static_cast<size_t>(rows) * (K / 2);
+}
+
+size_t svdq_scales_bytes(svdq_format f, int rows, int K) {
+  if (rows < 1 || K < 64 || K % 64) return 0;
+  if (f == SVDQ_NVFP4_G16) return pad128(rows) * (K / 16);
+  if (f == SVDQ_INT4_G64) return pad128(rows) * (K / 64) * 2;
+  return 0;
+}
+
+size_t awq_qweight_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 2);
+}
+
+size_t awq_sz_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return (static_cast<size_t>(N) + 15) / 16 * 16 * (K / 64) * 4;
+}
+
+int svdq_xl1_splits(int M, int K, int r) {
+  if (M < 1 || K < 64 || K % 64 || !rank_ok(r)) return 0;
+  return r == 0 ? 1 : qa_splits(M, K);
+}
+
+svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const void* X, int ldx,
+                              const float* smooth_inv, const void* L1s, void* codes,
+                              void* scales, float* xl1, svdq_stream_t stream) {
+  return quantize_act_impl(format, M, K, r, X, ldx, smooth_inv, L1s, codes, scales, xl1, false,
+                           stream);
+}
+
+svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, const void* X,
+                                      int ldx, const float* smooth_inv, const void* L1s,
+                                      void* codes, void* scales, float* xl1,
+                                      svdq_stream_t stream) {
+  return quantize_act_impl(format, M, K, r, X, ldx, smooth_inv, L1s, codes, scales, xl1, true,
+                           stream);
 }
 
 svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,

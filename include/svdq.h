@@ -131,6 +131,28 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
                               void* scales, float* xl1, svdq_stream_t stream);
 
 /*
+ * svdq_quantize_act_noalloc -- svdq_quantize_act with no working space from the
+ * caller: xl1 is only float32 [M, r] (same contents on return), and the partial
+ * down-projections of K splits 1 .. S-1 go to a working array the library
+ * holds in device memory for each device (one static array of 2^21 float32,
+ * 8 MiB; nothing is allocated or freed at any time). The pages describe no
+ * counterpart of this call: it exists for callers that must not hand the
+ * library any memory beyond the inputs and outputs.
+ *
+ * Limit: (S - 1) * M * r <= 2^21 with S = svdq_xl1_splits(M, K, r); a larger
+ * request returns SVDQ_ERR_UNSUPPORTED before anything is launched (r == 0 always
+ * fits). Nothing in the array needs to start at zero: each call writes every
+ * element it reads. The array is shared by all calls on a device, so two of
+ * these calls in flight at the same time (e.g. on different streams) race;
+ * calls ordered on one stream do not. Other arguments, layouts and errors as
+ * for svdq_quantize_act.
+ */
+svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, const void* X,
+                                      int ldx, const float* smooth_inv, const void* L1s,
+                                      void* codes, void* scales, float* xl1,
+                                      svdq_stream_t stream);
+
+/*
  * svdq_w4a4_linear -- steps a5..a6: the 4-bit GEMM with the low-rank
  * up-projection and bias accumulated into the same tensor-memory accumulator
  * (Nunchaku README, "Engine design" (b): the up projection and the 4-bit
