@@ -271,6 +271,29 @@ def run_reference(args, rank: int) -> None:
     }), flush=True)
 
 
+# ------------------------------------------------------------- multi-rank host logic
+def rank_rows(x_bits: np.ndarray, rank: int) -> np.ndarray:
+    """This rank's token batch (weak scaling: every rank has its own M rows):
+    the workload's rows rotated by 37 per rank, so ranks never share a batch."""
+    return x_bits if rank == 0 else np.roll(x_bits, 37 * rank, axis=0)
+
+
+def max_over_ranks(values, world: int, device) -> list:
+    """Every rank's per-step times -> their maxima over ranks (the slowest
+    rank defines the job's step time). world == 1 returns the values."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks over the (max-over-ranks) step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def config_block(n_gpus: int) -> dict:
     return {"workload": f"{SHAPE.name}: SVDQ W4A4 linear M={SHAPE.M} K={SHAPE.K} N={SHAPE.N} "
                         f"r={SHAPE.r} NVFP4 g16 + bias; AWQ W4A16 M={AWQ.M} K={AWQ.K} N={AWQ.N} g64",
@@ -315,7 +338,7 @@ def main() -> None:
 
     # ---------------------------------------------------------------- inputs
     d = WL.svdq_inputs(SHAPE)
-    x_bits = d["X"] if rank == 0 else np.roll(d["X"], 37 * rank, axis=0)
+    x_bits = rank_rows(d["X"], rank)
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
     X = to_dev(x_bits)
     W = to_dev(d["W"])
@@ -409,10 +432,7 @@ def main() -> None:
     del Y_host
 
     # ------------------------------------------------- max over ranks
-    t = torch.tensor([step_ms / args.steps, e2e_ms, k2_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step, ms_e2e, ms_k2 = (float(v) for v in t.cpu())
+    ms_step, ms_e2e, ms_k2 = max_over_ranks([step_ms / args.steps, e2e_ms, k2_ms], world, dev)
 
     # ------------------------------------------------- context: cuBLAS bf16
     cublas_tflops = None
@@ -453,7 +473,7 @@ def main() -> None:
     fp4_peak = bf16_peak * FP4_OVER_BF16
     k2_flops = 2.0 * M * N * K
     achieved = k2_flops / (ms_k2 * 1e-3) / 1e12
-    value = step_flops() * world / (ms_step * 1e-3) / 1e12
+    value = job_tflops(step_flops(), world, ms_step)
     traffic = recorded_traffic("w4a4_nvfp4_gemm_kernel")
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -466,7 +486,7 @@ def main() -> None:
                      "peak_note": f"{peaks['source']} bf16 {peak_kind} x {FP4_OVER_BF16:g} "
                                   f"(nominal FP4/BF16); vs nominal 9 PFLOP/s: {achieved / 9000:.3f}"},
         "cpu_baseline": cpu,
-        "e2e": {"value": step_flops() * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": job_tflops(step_flops(), world, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2 + Xa.numel() * 2,
                 "d2h_bytes_per_step": Y.numel() * 2 + Ya.numel() * 2, "ms_per_step": ms_e2e},
         "gpu_launches": 3 * args.steps,
