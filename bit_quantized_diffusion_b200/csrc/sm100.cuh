@@ -173,6 +173,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Arrive on another CTA's mbarrier (shared::cluster address) with CTA-scope
+// release: enough when the arrival hands over no memory contents, e.g. "these
+// tensor-memory columns have been read" (tcgen05.ld + wait::ld completed and a
+// tcgen05.fence::before_thread_sync issued before the arrival). Much cheaper
+// than the cluster-scope release below, which also waits for this thread's
+// outstanding writes.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (possibly another CTA's).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");

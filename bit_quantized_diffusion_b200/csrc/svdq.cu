@@ -386,10 +386,11 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
     return launch_int4_gemm(d, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, Y,
                             ldy, out, static_cast<cudaStream_t>(stream));
 
-  // CTA pairs (cta_group::2, 256-row tiles) pay off only when the K loop is long
-  // enough to hide their cross-CTA barrier traffic: measured on B200, single
-  // CTAs win at K = 3072 (with or without the low-rank branch), pairs at K >= 8192.
-  const bool pair_auto = K >= 8192;
+  // CTA pairs (cta_group::2, 256-row tiles): each CTA stages half of B, so a
+  // pair moves a third less operand data per MMA than two single CTAs; measured
+  // on B200 they are faster at every shape once the pair's cross-CTA arrivals
+  // use CTA-scope release (QKV 70.3 vs 75.0 us, fc1 r=128 115.8 vs 122.1 us).
+  const bool pair_auto = true;
   const bool pair = (d->gemm_pair_mode < 0 ? pair_auto : d->gemm_pair_mode != 0) && M > kGmBM;
   const int ctas = pair ? 2 : 1;
   const int b_rows = kGmBN / ctas;

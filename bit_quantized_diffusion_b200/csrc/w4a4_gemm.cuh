@@ -327,7 +327,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (kPair) mbar_arrive_cluster(lead(bar_ready(s)));
+          // The leader's pair MMA reads this CTA's rows through this SM's own
+          // tensor core from this CTA's shared memory: the writes above are
+          // ordered for it by the proxy fence and a CTA-scope release.
+          if (kPair) mbar_arrive_remote(lead(bar_ready(s)));
           else mbar_arrive(bar_ready(s));
         }
       }
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
-            if (kPair) mbar_arrive_cluster(free_bar);
+            if (kPair) mbar_arrive_remote(free_bar);  // hands over no memory contents
             else mbar_arrive(free_bar);
           }
         }
