@@ -18,30 +18,27 @@
 // bf16 pattern 0x4300 is the exact bf16 pair (128 + q), so the dequantization
 // is one mask per pair; the zero point enters once per group through xs.
 //
-// Persistent: one CTA per SM streams a contiguous run of 16-row blocks. Its
-// producer warp bulk-copies each block's weights and (scale, zero) pairs (up
-// to 48 groups per ring stage; a block of more groups spans several stages)
-// through a ring in shared memory, starting at once; meanwhile the sixteen
-// consumer warps stage X and the token sums xs. X rows are 16 bytes longer
-// than K and, inside every 64-wide group, hold a lane's B fragments for the
-// group's four K steps as 32 contiguous bytes (lane quad t: words t and t + 4
-// of each 16-element step), so a lane reads them with two 16-byte loads and
-// the 8 token rows fall in distinct banks. Consumer warp w takes the w-th
-// sixteenth of every stage's groups, each group's four MMAs as two independent
-// accumulation chains. After a block's last stage each consumer drops its
-// partial sums into a slot of a small ring and moves on; a reducer warp adds
-// the sixteen partials of each block in a fixed order and writes Y, so no
-// consumer ever waits for another.
+// Persistent: one CTA per SM owns a contiguous run of 16-row blocks and takes
+// them BPR at a time ("rounds"; BPR = 1, 2, 4 or 8, chosen by the host so the
+// sixteen consumer warps have work). Each block of a round gets 16 / BPR
+// consumer warps. A ring stage holds one slice of K for all the round's blocks,
+// 3 groups per warp, so every warp handles exactly three groups per stage (all
+// loads first, then two MMA chains per group). A producer warp fills each stage
+// with two tiled TMA copies (fragment-ordered weights and (s, z) pairs, as 3-D
+// boxes over blocks x groups), starting at kernel entry, while the consumers stage X in
+// shared memory in B-fragment order and the per-group token sums xs. Each warp
+// keeps its block's partial sum in registers for the whole round; at the end of
+// the round the block's first warp adds the block's partials in warp order and
+// writes Y.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace svdq {
 
-constexpr int kAwqConsumers = 16;                         // warps sharing each block (K split)
-constexpr int kAwqThreads = 32 * (kAwqConsumers + 2);     // + producer and reducer warps
-constexpr int kAwqRedSlots = 4;                           // blocks of partial sums in flight
-constexpr int kAwqStageGroups = 48;                       // groups per ring stage at most
+constexpr int kAwqConsumers = 16;                         // consumer warps
+constexpr int kAwqThreads = 32 * (kAwqConsumers + 1);     // + the producer warp
+constexpr int kAwqWarpGroups = 3;                         // groups per warp per ring stage
 constexpr int kAwqGroupBytes = 512 + 64;                  // fragment words + (s, z) of 16 rows
 constexpr int kAwqMaxStages = 4;
 constexpr int kAwqMaxM = 64;
@@ -49,6 +46,7 @@ constexpr int kAwqMaxM = 64;
 struct AwqParams {
   int M, N, K;
   int stages;             // ring depth (2..4)
+  int bpr;                // blocks per round: 1, 2, 4 or 8
   const __nv_bfloat16* X;
   const uint4* qweight;   // fragment order
   const uint32_t* sz;     // (s, z) bf16 pairs
@@ -57,22 +55,20 @@ struct AwqParams {
   uint32_t* status;
 };
 
-// dynamic shared memory: ring, X rows, token sums, reduction buffer, barriers
-__host__ __device__ constexpr int awq_stage_groups(int K) {
-  return K / 64 < kAwqStageGroups ? K / 64 : kAwqStageGroups;
-}
-__host__ __device__ constexpr size_t awq_stage_bytes(int K) {
-  return static_cast<size_t>(awq_stage_groups(K)) * kAwqGroupBytes;
+// dynamic shared memory: ring, X rows, token sums, partial sums, barriers.
+// A stage holds kAwqConsumers * kAwqWarpGroups groups (for any blocks per round).
+__host__ __device__ constexpr size_t awq_stage_bytes() {
+  return static_cast<size_t>(kAwqConsumers) * kAwqWarpGroups * kAwqGroupBytes;  // 27 KB
 }
 __host__ __device__ constexpr size_t awq_xrow_bytes(int K) { return static_cast<size_t>(K) * 2 + 16; }
 __host__ __device__ constexpr size_t awq_fixed_bytes(int M, int K, int kMB) {
   return static_cast<size_t>(M + 1) * awq_xrow_bytes(K) +               // X
          static_cast<size_t>(kMB) * 8 * (K / 64) * 4 +                  // xs
-         static_cast<size_t>(kAwqRedSlots) * kAwqConsumers * 32 * 4 * kMB * 4 +  // partial sums
-         8 * 2 * (kAwqMaxStages + kAwqRedSlots) + 128;                  // barriers, alignment
+         static_cast<size_t>(kAwqConsumers) * 32 * 4 * kMB * 4 +        // partial sums
+         8 * 2 * kAwqMaxStages + 128;                                   // barriers, alignment
 }
 __host__ __device__ constexpr size_t awq_smem_bytes(int M, int K, int kMB, int stages) {
-  return static_cast<size_t>(stages) * awq_stage_bytes(K) + awq_fixed_bytes(M, K, kMB);
+  return static_cast<size_t>(stages) * awq_stage_bytes() + awq_fixed_bytes(M, K, kMB);
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -214,42 +210,44 @@ __device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint
   }
 }
 
+// tm_q: qweight as [N/16 blocks][K/64 groups][64 x 8 bytes]; tm_sz: (s, z) pairs as
+// [N/16][K/64][8 x 8 bytes]: one box {64 or 8, GSK, BPR} is one stage's slice of
+// the round's blocks (rows past N and groups past K arrive as zeros).
 template <int kMB>  // number of 8-token blocks (1 or 2; the host splits larger M)
-__global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParams p) {
+__global__ void __launch_bounds__(kAwqThreads, 1)
+    awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sz,
+                    const AwqParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~uintptr_t(127));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.K / 64;
-  const int GS = awq_stage_groups(p.K);
-  const int nst = (G + GS - 1) / GS;                 // ring stages per block
+  const int BPR = p.bpr;                               // blocks per round
+  const int WPB = kAwqConsumers / BPR;                 // warps per block
+  const int GSK = kAwqWarpGroups * WPB;                // groups per block per stage
+  const int nst = (G + GSK - 1) / GSK;                 // ring stages per round
   const int NS = p.stages;
-  const size_t SB = awq_stage_bytes(p.K);
+  const size_t SB = awq_stage_bytes();
+  const uint32_t sz_off = static_cast<uint32_t>(BPR) * GSK * 512;  // (s, z) part of a stage
   const int nblocks = (p.N + 15) / 16;
   const int b_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * nblocks / gridDim.x);
   const int b_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * nblocks / gridDim.x);
+  const int nrounds = (b_end - b_begin + BPR - 1) / BPR;
   const int r0 = lane >> 2, c0 = 2 * (lane & 3);
 
   uint8_t* ring = smem;
   const size_t xrow_bytes = awq_xrow_bytes(p.K);
   uint8_t* xsm = ring + NS * SB;  // [M + 1][K + 8] bf16, row M all zero
   float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M + 1) * xrow_bytes);  // [kMB*8][G]
-  constexpr int kSlot = kAwqConsumers * 32 * 4 * kMB;  // floats per partial-sum slot
-  float* red = xs + kMB * 8 * G;                     // [slots][consumers][32][4 kMB]
-  const uint32_t bars = (smem_u32(red + kAwqRedSlots * kSlot) + 7) & ~7u;
+  float* red = xs + kMB * 8 * G;                     // [consumers][32][4 kMB]
+  const uint32_t bars = (smem_u32(red + kAwqConsumers * 32 * 4 * kMB) + 7) & ~7u;
   auto full = [&](int s) { return bars + 8 * s; };
   auto empty = [&](int s) { return bars + 8 * (kAwqMaxStages + s); };
-  auto red_full = [&](int q) { return bars + 8 * (2 * kAwqMaxStages + q); };
-  auto red_empty = [&](int q) { return bars + 8 * (2 * kAwqMaxStages + kAwqRedSlots + q); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), kAwqConsumers);
-    }
-    for (int q = 0; q < kAwqRedSlots; ++q) {
-      mbar_init(red_full(q), kAwqConsumers);
-      mbar_init(red_empty(q), 1);
     }
     fence_barrier_init();
   }
@@ -260,56 +258,22 @@ __global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParam
     if (elect_one()) {
       int it = 0;
       bool ok = true;
-      for (int b = b_begin; b < b_end && ok; ++b) {
+      for (int rr = 0; rr < nrounds && ok; ++rr) {
+        const int bb = b_begin + rr * BPR;
         for (int t = 0; t < nst && ok; ++t, ++it) {
           const int s = it % NS;
-          // the producer and the reducer are not on the critical path: they
-          // wait suspended, leaving the issue slots to the consumers
+          // the producer is not on the critical path: it waits suspended
           ok = mbar_wait(empty(s), ((it / NS) & 1) ^ 1, p.status, kWaitLimitNs, 2000u);
           if (!ok) break;
-          const int g0 = t * GS, n = min(GS, G - g0);
-          const size_t bg = static_cast<size_t>(b) * G + g0;
           const uint32_t dst = smem_u32(ring + s * SB);
-          mbar_arrive_expect_tx(full(s), n * kAwqGroupBytes);
-          bulk_load(dst, p.qweight + bg * 32, n * 512, full(s));
-          bulk_load(dst + GS * 512, p.sz + bg * 16, n * 64, full(s));
+          // two tiled copies fill the stage; their boxes count in full
+          mbar_arrive_expect_tx(full(s), BPR * GSK * kAwqGroupBytes);
+          tma_load_3d(dst, &tm_q, full(s), 0, t * GSK, bb);
+          tma_load_3d(dst + sz_off, &tm_sz, full(s), 0, t * GSK, bb);
         }
       }
     }
     return;  // the consumers synchronise among themselves from here on
-  }
-  if (warp == kAwqConsumers + 1) {
-    // ------------------------------------------------------------ reducer
-    for (int b = b_begin; b < b_end; ++b) {
-      const int jj = b - b_begin, q = jj % kAwqRedSlots;
-      const bool ok = mbar_wait(red_full(q), (jj / kAwqRedSlots) & 1, p.status, kWaitLimitNs, 2000u);
-      const float* rb = red + q * kSlot;
-#pragma unroll
-      for (int mb = 0; mb < kMB; ++mb) {
-        float4 v = *reinterpret_cast<const float4*>(rb + (lane * kMB + mb) * 4);
-#pragma unroll
-        for (int w = 1; w < kAwqConsumers; ++w) {
-          const float4 u = *reinterpret_cast<const float4*>(rb + ((w * 32 + lane) * kMB + mb) * 4);
-          v.x += u.x;
-          v.y += u.y;
-          v.z += u.z;
-          v.w += u.w;
-        }
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int n = b * 16 + r0 + ((j & 2) ? 8 : 0);
-          const int m = mb * 8 + c0 + (j & 1);
-          if (ok && n < p.N && m < p.M) {
-            const float bb = p.bias != nullptr ? __bfloat162float(p.bias[n]) : 0.0f;
-            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(vv[j] + bb);
-          }
-        }
-      }
-      __syncwarp();  // all lanes have read the slot
-      if (lane == 0) mbar_arrive(red_empty(q));
-    }
-    return;
   }
 
   // -------------------------------------------------------------- consumers
@@ -317,48 +281,47 @@ __global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParam
   // X in shared memory, plus one zero row that padding tokens read. Source
   // 16-byte unit c of a row holds words 4h..4h+3 (h = c % 2) of K step
   // ks = (c / 2) % 4 of group c / 8; word 4h + t goes to lane quad t's run.
-  // Eight loads per thread are issued before any store, so their latencies overlap.
-  const int units = (p.M + 1) * (p.K / 8);
-  for (int t0 = threadIdx.x; t0 < units; t0 += 8 * kCT) {
-    uint4 v[8];
+  // A thread owns unit columns c = tid, tid + 512, ...; its rows' loads are
+  // issued four at a time before their stores, so their latencies overlap.
+  const int U = p.K / 8;  // 16-byte units per row
+  for (int c = threadIdx.x; c < U; c += kCT) {
+    const int ks = (c >> 1) & 3, h = c & 1;
+    const uint4* src = reinterpret_cast<const uint4*>(p.X) + c;
+    uint8_t* dst = xsm + (c >> 3) * 128;
+    for (int m0 = 0; m0 <= p.M; m0 += 4) {
+      uint4 v[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int t = t0 + u * kCT;
-      const int m = t / (p.K / 8), c = t % (p.K / 8);
-      v[u] = (t < units && m < p.M)
-                 ? __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(m) * p.K) + c)
-                 : make_uint4(0u, 0u, 0u, 0u);
-    }
+      for (int u = 0; u < 4; ++u)
+        v[u] = m0 + u < p.M ? __ldg(src + static_cast<size_t>(m0 + u) * U) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int t = t0 + u * kCT;
-      if (t >= units) break;
-      const int m = t / (p.K / 8), c = t % (p.K / 8);
-      uint32_t* grp = reinterpret_cast<uint32_t*>(xsm + m * xrow_bytes + (c / 8) * 128);
-      const int ks = (c / 2) % 4, h = c % 2;
-      grp[0 * 8 + ks * 2 + h] = v[u].x;
-      grp[1 * 8 + ks * 2 + h] = v[u].y;
-      grp[2 * 8 + ks * 2 + h] = v[u].z;
-      grp[3 * 8 + ks * 2 + h] = v[u].w;
+      for (int u = 0; u < 4; ++u) {
+        if (m0 + u > p.M) break;
+        uint32_t* grp = reinterpret_cast<uint32_t*>(dst + (m0 + u) * xrow_bytes);
+        grp[0 * 8 + ks * 2 + h] = v[u].x;
+        grp[1 * 8 + ks * 2 + h] = v[u].y;
+        grp[2 * 8 + ks * 2 + h] = v[u].z;
+        grp[3 * 8 + ks * 2 + h] = v[u].w;
+      }
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   // per-group token sums xs[m][g] (rows >= M are zero)
-  for (int t = threadIdx.x; t < kMB * 8 * G; t += kCT) {
-    const int m = t / G, g = t % G;
-    float sum = 0.0f;
-    if (m < p.M) {
-      const uint4* xp = reinterpret_cast<const uint4*>(xsm + m * xrow_bytes + g * 128);
+  for (int g = threadIdx.x; g < G; g += kCT) {
+    for (int m = 0; m < kMB * 8; ++m) {
+      float sum = 0.0f;
+      if (m < p.M) {
+        const uint4* xq = reinterpret_cast<const uint4*>(xsm + m * xrow_bytes + g * 128);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 v = xp[j];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = xq[j];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+          for (int e = 0; e < 4; ++e)
+            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+        }
       }
+      xs[m * G + g] = sum;
     }
-    xs[t] = sum;
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 
@@ -371,10 +334,13 @@ __global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParam
     xa[mb] = smem_u32(xsm) + (m < p.M ? m : p.M) * static_cast<uint32_t>(xrow_bytes) + (lane & 3) * 32;
   }
   const uint32_t xs_a = smem_u32(xs) + c0 * G * 4;  // xs[c0][0]
+  const int jslot = warp / WPB, part = warp % WPB;  // this warp's block slot and K share
   bool ok = true;
   int s = 0;          // ring slot
   uint32_t ph = 0;    // its phase parity
-  for (int b = b_begin; b < b_end; ++b) {
+  for (int rr = 0; rr < nrounds; ++rr) {
+    const int b = b_begin + rr * BPR + jslot;
+    const bool active = b < b_end;
     float acc[kMB][4];
 #pragma unroll
     for (int mb = 0; mb < kMB; ++mb)
@@ -382,16 +348,19 @@ __global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParam
       for (int j = 0; j < 4; ++j) acc[mb][j] = 0.0f;
     for (int t = 0; t < nst; ++t) {
       if (ok) ok = mbar_wait_poll(full(s), ph, p.status);
-      const int g0 = t * GS, n = min(GS, G - g0);
-      const int lo = warp * n / kAwqConsumers, hi = (warp + 1) * n / kAwqConsumers;
+      const int g0 = t * GSK, n = min(GSK, G - g0);
+      // a full stage gives every warp kAwqWarpGroups groups; only a last, partial
+      // stage needs the general split
+      const int lo = n == GSK ? part * kAwqWarpGroups : part * n / WPB;
+      const int hi = n == GSK ? lo + kAwqWarpGroups : (part + 1) * n / WPB;
       const uint32_t st = smem_u32(ring + s * SB);
-      const uint32_t wp = st + lo * 512 + lane * 16;           // this lane's fragment word
-      const uint32_t szp = st + GS * 512 + lo * 64 + r0 * 4;   // (s, z) of row r0
-      const uint32_t xo = (g0 + lo) * 128;                     // group offset in the X runs
-      const uint32_t xsp = xs_a + (g0 + lo) * 4;               // xs[c0][g]
-      if (ok) {
-        if (kMB == 1 && hi - lo == 3) {
-          awq_groups<kMB, 3>(wp, szp, xa, xo, xsp, G, acc);   // 48-group stages: 3 per warp
+      const uint32_t wp = st + jslot * GSK * 512 + lo * 512 + lane * 16;     // fragment word
+      const uint32_t szp = st + sz_off + jslot * GSK * 64 + lo * 64 + r0 * 4;  // (s, z) of row r0
+      const uint32_t xo = (g0 + lo) * 128;                                    // X run offset
+      const uint32_t xsp = xs_a + (g0 + lo) * 4;                              // xs[c0][g]
+      if (ok && active) {
+        if (hi - lo == kAwqWarpGroups) {
+          awq_groups<kMB, kAwqWarpGroups>(wp, szp, xa, xo, xsp, G, acc);
         } else {
           for (int j = 0; j < hi - lo; ++j)
             awq_groups<kMB, 1>(wp + j * 512, szp + j * 64, xa, xo + j * 128, xsp + j * 4, G, acc);
@@ -404,16 +373,37 @@ __global__ void __launch_bounds__(kAwqThreads, 1) awq_gemv_kernel(const AwqParam
         ph ^= 1u;
       }
     }
-    // hand this warp's partial sums of the block to the reducer
-    const int jj = b - b_begin, q = jj % kAwqRedSlots;
-    if (ok) ok = mbar_wait_poll(red_empty(q), ((jj / kAwqRedSlots) & 1) ^ 1, p.status);
-    float* rb = red + q * kSlot;
+    // the block's partial sums (one per K share), added in share order by share 0
 #pragma unroll
     for (int mb = 0; mb < kMB; ++mb)
-      *reinterpret_cast<float4*>(rb + ((warp * 32 + lane) * kMB + mb) * 4) =
+      *reinterpret_cast<float4*>(red + ((warp * 32 + lane) * kMB + mb) * 4) =
           make_float4(acc[mb][0], acc[mb][1], acc[mb][2], acc[mb][3]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(red_full(q));
+    asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+    if (part == 0 && active && ok) {
+#pragma unroll
+      for (int mb = 0; mb < kMB; ++mb) {
+        float4 v = *reinterpret_cast<const float4*>(red + ((warp * 32 + lane) * kMB + mb) * 4);
+        for (int q = 1; q < WPB; ++q) {
+          const float4 u =
+              *reinterpret_cast<const float4*>(red + (((warp + q) * 32 + lane) * kMB + mb) * 4);
+          v.x += u.x;
+          v.y += u.y;
+          v.z += u.z;
+          v.w += u.w;
+        }
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = b * 16 + r0 + ((j & 2) ? 8 : 0);
+          const int m = mb * 8 + c0 + (j & 1);
+          if (n < p.N && m < p.M) {
+            const float bb = p.bias != nullptr ? __bfloat162float(p.bias[n]) : 0.0f;
+            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(vv[j] + bb);
+          }
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");  // red is free for the next round
   }
 }
 

@@ -167,6 +167,25 @@ bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint6
   return r == CUDA_SUCCESS;
 }
 
+// A 3-D map over [outer][mid][inner] 8-byte elements, rows contiguous, for
+// unswizzled boxes {inner, box_mid, box_outer} (the inner dimension whole).
+bool make_tmap_3d_u64(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer,
+                      uint32_t box_mid, uint32_t box_outer) {
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner * 8, inner * 8 * mid};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), box_mid, box_outer};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "svdq: 3-d tensor map (%llu x %llu x %llu) failed: %d\n",
+                 static_cast<unsigned long long>(inner), static_cast<unsigned long long>(mid),
+                 static_cast<unsigned long long>(outer), static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
 bool rank_ok(int r) { return r == 0 || (r % 16 == 0 && r >= 16 && r <= 256); }
 
 size_t pad128(int rows) { return (static_cast<size_t>(rows) + 127) / 128 * 128; }
@@ -476,8 +495,18 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
   while (mc > 1 && !fits(mc, 2)) --mc;
   if (!fits(mc, 2)) return SVDQ_ERR_UNSUPPORTED;
   const int nblocks = (N + 15) / 16;
-  // one persistent CTA per SM, each streaming a contiguous run of 16-row blocks
+  // one persistent CTA per SM, each streaming a contiguous run of 16-row blocks,
+  // taken bpr at a time: the smallest power of two (<= 8) covering its blocks
   const int grid = nblocks < d->num_sms ? nblocks : d->num_sms;
+  const int per_cta = (nblocks + grid - 1) / grid;
+  int bpr = 1;
+  while (bpr < per_cta && bpr < 8) bpr *= 2;
+  // the stage boxes: weights [blocks][groups][64 x 8 B], (s, z) [blocks][groups][8 x 8 B]
+  const int G = K / 64, wpb = kAwqConsumers / bpr, gsk = kAwqWarpGroups * wpb;
+  CUtensorMap tm_q, tm_sz;
+  if (!make_tmap_3d_u64(&tm_q, qweight, 64, G, nblocks, gsk, bpr) ||
+      !make_tmap_3d_u64(&tm_sz, sz, 8, G, nblocks, gsk, bpr))
+    return SVDQ_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int m0 = 0; m0 < M; m0 += mc) {
     const int mm = M - m0 < mc ? M - m0 : mc;
@@ -489,6 +518,7 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
     p.N = N;
     p.K = K;
     p.stages = stages;
+    p.bpr = bpr;
     p.X = static_cast<const __nv_bfloat16*>(X) + static_cast<size_t>(m0) * K;
     p.qweight = static_cast<const uint4*>(qweight);
     p.sz = static_cast<const uint32_t*>(sz);
@@ -497,9 +527,9 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
     p.status = d->status;
     const size_t smem = awq_smem_bytes(mm, K, kmb, stages);
     if (kmb == 1)
-      awq_gemv_kernel<1><<<grid, kAwqThreads, smem, s>>>(p);
+      awq_gemv_kernel<1><<<grid, kAwqThreads, smem, s>>>(tm_q, tm_sz, p);
     else
-      awq_gemv_kernel<2><<<grid, kAwqThreads, smem, s>>>(p);
+      awq_gemv_kernel<2><<<grid, kAwqThreads, smem, s>>>(tm_q, tm_sz, p);
   }
   return launch_status();
 }
