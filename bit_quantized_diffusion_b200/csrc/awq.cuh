@@ -22,11 +22,11 @@
 // them BPR at a time ("rounds"; BPR = 1, 2, 4 or 8, chosen by the host so the
 // sixteen consumer warps have work). Each block of a round gets 16 / BPR
 // consumer warps. A ring stage holds one slice of K for all the round's blocks,
-// 3 groups per warp, so every warp handles exactly three groups per stage (all
+// 4 groups per warp, so every warp handles exactly four groups per stage (all
 // loads first, then two MMA chains per group). A producer warp fills each stage
 // with two tiled TMA copies (fragment-ordered weights and (s, z) pairs, as 3-D
 // boxes over blocks x groups), starting at kernel entry, while the consumers stage X in
-// shared memory in B-fragment order and the per-group token sums xs. Each warp
+// shared memory in B-fragment order, summing each group's tokens (xs) on the way. Each warp
 // keeps its block's partial sum in registers for the whole round; at the end of
 // the round the block's first warp adds the block's partials in warp order and
 // writes Y.
@@ -38,7 +38,7 @@ namespace svdq {
 
 constexpr int kAwqConsumers = 16;                         // consumer warps
 constexpr int kAwqThreads = 32 * (kAwqConsumers + 1);     // + the producer warp
-constexpr int kAwqWarpGroups = 3;                         // groups per warp per ring stage
+constexpr int kAwqWarpGroups = 4;                         // groups per warp per ring stage
 constexpr int kAwqGroupBytes = 512 + 64;                  // fragment words + (s, z) of 16 rows
 constexpr int kAwqMaxStages = 4;
 constexpr int kAwqMaxM = 64;
@@ -61,9 +61,12 @@ __host__ __device__ constexpr size_t awq_stage_bytes() {
   return static_cast<size_t>(kAwqConsumers) * kAwqWarpGroups * kAwqGroupBytes;  // 27 KB
 }
 __host__ __device__ constexpr size_t awq_xrow_bytes(int K) { return static_cast<size_t>(K) * 2 + 16; }
+// Row stride of the token sums xs (floats): the group count rounded up to
+// 4 (mod 32), so the tokens 0, 2, 4, 6 a lane quad reads hit different banks.
+__host__ __device__ constexpr int awq_xs_ld(int K) { return (K / 64 + 27) / 32 * 32 + 4; }
 __host__ __device__ constexpr size_t awq_fixed_bytes(int M, int K, int kMB) {
   return static_cast<size_t>(M + 1) * awq_xrow_bytes(K) +               // X
-         static_cast<size_t>(kMB) * 8 * (K / 64) * 4 +                  // xs
+         static_cast<size_t>(kMB) * 8 * awq_xs_ld(K) * 4 +               // xs
          static_cast<size_t>(kAwqConsumers) * 32 * 4 * kMB * 4 +        // partial sums
          8 * 2 * kAwqMaxStages + 128;                                   // barriers, alignment
 }
@@ -78,6 +81,16 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       " {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator: the first K step of a chain.
+__device__ __forceinline__ void mma_bf16_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                 uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32"
+      " {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -135,10 +148,10 @@ __device__ __forceinline__ void awq_dequant_word(uint32_t w, uint32_t (&a)[4]) {
 //   wp   this lane's first fragment word          (+512 per group)
 //   szp  (s, z) of row r0 of the first group        (+64 per group, row r0 + 8 at +32)
 //   xa   this lane's X fragment runs, xo the first group's offset in them (+128 per group)
-//   xsp  xs[c0][first group]                        (+4 per group, token c0 + 1 at +4 G)
+//   xsp  xs[c0][first group]                        (+4 per group, token c0 + 1 at +4 xs_ld)
 template <int kMB, int kN>  // kN <= 4
 __device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint32_t (&xa)[kMB],
-                                           uint32_t xo, uint32_t xsp, int G, float (&acc)[kMB][4]) {
+                                           uint32_t xo, uint32_t xsp, int xs_ld, float (&acc)[kMB][4]) {
   uint4 w[kN], xl[kN][kMB][2];
   uint32_t sz0[kN], sz8[kN];
   float xs0[kN][kMB], xs1[kN][kMB];
@@ -146,8 +159,8 @@ __device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint
 #pragma unroll
   for (int mb = 0; mb < kMB; ++mb) {
     xb[mb] = xa[mb] + xo;
-    xs0a[mb] = xsp + mb * 8 * G * 4;
-    xs1a[mb] = xs0a[mb] + G * 4;
+    xs0a[mb] = xsp + mb * 8 * xs_ld * 4;
+    xs1a[mb] = xs0a[mb] + xs_ld * 4;
   }
 #pragma unroll
   for (int u = 0; u < kN; ++u) {
@@ -174,14 +187,6 @@ __device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint
   }
   float pc[kN][2][kMB][4];
 #pragma unroll
-  for (int u = 0; u < kN; ++u)
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int mb = 0; mb < kMB; ++mb)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pc[u][c][mb][e] = 0.0f;
-#pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
     for (int u = 0; u < kN; ++u) {
@@ -191,7 +196,10 @@ __device__ __forceinline__ void awq_groups(uint32_t wp, uint32_t szp, const uint
 #pragma unroll
       for (int mb = 0; mb < kMB; ++mb) {
         const uint4& x = xl[u][mb][ks >> 1];
-        mma_bf16_16816(pc[u][ks & 1][mb], a, (ks & 1) ? x.z : x.x, (ks & 1) ? x.w : x.y);
+        if (ks < 2)
+          mma_bf16_16816_z(pc[u][ks & 1][mb], a, (ks & 1) ? x.z : x.x, (ks & 1) ? x.w : x.y);
+        else
+          mma_bf16_16816(pc[u][ks & 1][mb], a, (ks & 1) ? x.z : x.x, (ks & 1) ? x.w : x.y);
       }
     }
   }
@@ -238,8 +246,9 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
   uint8_t* ring = smem;
   const size_t xrow_bytes = awq_xrow_bytes(p.K);
   uint8_t* xsm = ring + NS * SB;  // [M + 1][K + 8] bf16, row M all zero
-  float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M + 1) * xrow_bytes);  // [kMB*8][G]
-  float* red = xs + kMB * 8 * G;                     // [consumers][32][4 kMB]
+  float* xs = reinterpret_cast<float*>(xsm + static_cast<size_t>(p.M + 1) * xrow_bytes);  // [kMB*8][xs_ld]
+  const int xs_ld = awq_xs_ld(p.K);
+  float* red = xs + kMB * 8 * xs_ld;                 // [consumers][32][4 kMB]
   const uint32_t bars = (smem_u32(red + kAwqConsumers * 32 * 4 * kMB) + 7) & ~7u;
   auto full = [&](int s) { return bars + 8 * s; };
   auto empty = [&](int s) { return bars + 8 * (kAwqMaxStages + s); };
@@ -252,10 +261,12 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dep_launch();
 
   if (warp == kAwqConsumers) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
+      grid_dep_wait();
       int it = 0;
       bool ok = true;
       for (int rr = 0; rr < nrounds && ok; ++rr) {
@@ -278,13 +289,19 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
 
   // -------------------------------------------------------------- consumers
   constexpr int kCT = kAwqConsumers * 32;
+  grid_dep_wait();  // X and Y may be the previous grid's
   // X in shared memory, plus one zero row that padding tokens read. Source
   // 16-byte unit c of a row holds words 4h..4h+3 (h = c % 2) of K step
   // ks = (c / 2) % 4 of group c / 8; word 4h + t goes to lane quad t's run.
-  // A thread owns unit columns c = tid, tid + 512, ...; its rows' loads are
+  // Thread tid owns unit columns c = tid, tid + 512, ... (every thread takes
+  // every pass, so the shuffles below see full warps); its rows' loads are
   // issued four at a time before their stores, so their latencies overlap.
-  const int U = p.K / 8;  // 16-byte units per row
-  for (int c = threadIdx.x; c < U; c += kCT) {
+  // The eight units of a group sit in eight consecutive lanes: their sums,
+  // combined by a fixed xor tree, give the token sums xs[m][g].
+  const int U = p.K / 8;  // 16-byte units per row (a multiple of 8)
+  for (int c0 = 0; c0 < U; c0 += kCT) {
+    const int c = c0 + threadIdx.x;
+    const bool has = c < U;
     const int ks = (c >> 1) & 3, h = c & 1;
     const uint4* src = reinterpret_cast<const uint4*>(p.X) + c;
     uint8_t* dst = xsm + (c >> 3) * 128;
@@ -292,36 +309,36 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
       uint4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        v[u] = m0 + u < p.M ? __ldg(src + static_cast<size_t>(m0 + u) * U) : make_uint4(0u, 0u, 0u, 0u);
+        v[u] = has && m0 + u < p.M ? __ldg(src + static_cast<size_t>(m0 + u) * U) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        if (m0 + u > p.M) break;
-        uint32_t* grp = reinterpret_cast<uint32_t*>(dst + (m0 + u) * xrow_bytes);
-        grp[0 * 8 + ks * 2 + h] = v[u].x;
-        grp[1 * 8 + ks * 2 + h] = v[u].y;
-        grp[2 * 8 + ks * 2 + h] = v[u].z;
-        grp[3 * 8 + ks * 2 + h] = v[u].w;
+        const int m = m0 + u;
+        if (m > p.M) break;
+        if (has) {
+          uint32_t* grp = reinterpret_cast<uint32_t*>(dst + m * xrow_bytes);
+          grp[0 * 8 + ks * 2 + h] = v[u].x;
+          grp[1 * 8 + ks * 2 + h] = v[u].y;
+          grp[2 * 8 + ks * 2 + h] = v[u].z;
+          grp[3 * 8 + ks * 2 + h] = v[u].w;
+        }
+        if (m < p.M) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          float e[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) e[j] = __uint_as_float(w[j] << 16) + __uint_as_float(w[j] & 0xFFFF0000u);
+          float sum = (e[0] + e[1]) + (e[2] + e[3]);
+          sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+          sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+          sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+          if (has && (c & 7) == 0) xs[m * xs_ld + (c >> 3)] = sum;
+        }
       }
     }
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
-  // per-group token sums xs[m][g] (rows >= M are zero)
-  for (int g = threadIdx.x; g < G; g += kCT) {
-    for (int m = 0; m < kMB * 8; ++m) {
-      float sum = 0.0f;
-      if (m < p.M) {
-        const uint4* xq = reinterpret_cast<const uint4*>(xsm + m * xrow_bytes + g * 128);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = xq[j];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-      }
-      xs[m * G + g] = sum;
-    }
+  // token rows M .. 8 kMB - 1 are padding: their sums are zero
+  for (int i = threadIdx.x; i < (kMB * 8 - p.M) * G; i += kCT) {
+    const int m = p.M + i / G, g = i - (i / G) * G;
+    xs[m * xs_ld + g] = 0.0f;
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 
@@ -333,7 +350,7 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
     const int m = mb * 8 + r0;
     xa[mb] = smem_u32(xsm) + (m < p.M ? m : p.M) * static_cast<uint32_t>(xrow_bytes) + (lane & 3) * 32;
   }
-  const uint32_t xs_a = smem_u32(xs) + c0 * G * 4;  // xs[c0][0]
+  const uint32_t xs_a = smem_u32(xs) + c0 * xs_ld * 4;  // xs[c0][0]
   const int jslot = warp / WPB, part = warp % WPB;  // this warp's block slot and K share
   bool ok = true;
   int s = 0;          // ring slot
@@ -360,10 +377,10 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
       const uint32_t xsp = xs_a + (g0 + lo) * 4;                              // xs[c0][g]
       if (ok && active) {
         if (hi - lo == kAwqWarpGroups) {
-          awq_groups<kMB, kAwqWarpGroups>(wp, szp, xa, xo, xsp, G, acc);
+          awq_groups<kMB, kAwqWarpGroups>(wp, szp, xa, xo, xsp, xs_ld, acc);
         } else {
           for (int j = 0; j < hi - lo; ++j)
-            awq_groups<kMB, 1>(wp + j * 512, szp + j * 64, xa, xo + j * 128, xsp + j * 4, G, acc);
+            awq_groups<kMB, 1>(wp + j * 512, szp + j * 64, xa, xo + j * 128, xsp + j * 4, xs_ld, acc);
         }
       }
       __syncwarp();  // every lane is done with the stage before it is released

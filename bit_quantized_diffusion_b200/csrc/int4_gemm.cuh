@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  grid_dep_wait();  // the prologue above touches no global memory the previous grid may write
+  grid_dep_launch();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 

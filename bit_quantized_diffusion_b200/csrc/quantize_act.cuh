@@ -141,6 +141,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  grid_dep_wait();  // the prologue above touches no global memory the previous grid may write
+  grid_dep_launch();
   tc_fence_after();
   const uint32_t tmem_base = r > 0 ? *tmem_slot : 0;
 
@@ -352,6 +354,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
 // The K splits' partial down-projections, added in split order into split 0:
 // xl1 = ((xl1 + rest[0]) + ...) + rest[S-2]; n4 float4 per split.
 __global__ void xl1_reduce_kernel(float4* xl1, const float4* rest, int splits, size_t n4) {
+  grid_dep_wait();
+  grid_dep_launch();
   for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n4;
        t += static_cast<size_t>(gridDim.x) * blockDim.x) {
     float4 v = xl1[t];

@@ -143,6 +143,24 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// Programmatic dependent launch. grid_dep_wait blocks until the grid before
+// this one in the stream has completed and its memory operations are visible;
+// grid_dep_launch lets the grid after this one be scheduled now (it still runs
+// its own grid_dep_wait before touching this grid's results). Both are no-ops
+// for a grid launched without programmatic stream serialization.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Warm L2 with [src, src + bytes) (16-byte aligned, a multiple of 16 bytes);
+// no data reaches this SM and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int c0, int c1) {
   asm volatile(

@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/svdq.h"
 #include "awq.cuh"
@@ -39,6 +40,7 @@ struct DeviceInfo {
   int gemm_pair_mode = -1;  // -1: by shape; SVDQ_GEMM_PAIR=0/1 forces single-CTA / CTA-pair tiles
   uint32_t* status = nullptr;
   float* xl1_scratch = nullptr;  // device address of g_xl1_scratch
+  bool pdl = true;  // programmatic dependent launch of the hot-path kernels (SVDQ_PDL=0: off)
 };
 
 std::mutex g_mu;
@@ -49,6 +51,38 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+
+// Launch a hot-path kernel. With programmatic dependent launch the grid may be
+// scheduled while the previous grid in the stream is finishing: every such
+// kernel runs grid_dep_wait before its first global access, so stream order
+// holds, and only its launch and prologue overlap the previous grid's tail.
+// cluster_x > 1 launches clusters of that many CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(const DeviceInfo* d, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                          size_t smem, cudaStream_t stream, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (d->pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Per-device set-up (status word address, SM count, kernel attributes), done
 // once per device with that device current.
@@ -132,6 +166,7 @@ svdq_status device_setup(DeviceInfo** out) {
                      d.gemm_pairs);
     }
     if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) d.gemm_pair_mode = std::atoi(e) != 0;
+    if (const char* e = std::getenv("SVDQ_PDL")) d.pdl = std::atoi(e) != 0;
     d.status = static_cast<uint32_t*>(st);
     d.xl1_scratch = static_cast<float*>(scratch);
     d.ready = true;
@@ -235,8 +270,11 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
   p.tiles_m = (M + kI4BM - 1) / kI4BM;
   p.tiles = p.tiles_m * ((N + kI4BN - 1) / kI4BN);
   const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
-  w4a4_int4_gemm_kernel<<<grid, kI4Threads, kI4SmemBytes, stream>>>(tm_a, tm_b, tm_sa, tm_sw,
-                                                                     tm_l2, p);
+  if (launch_kernel(d, w4a4_int4_gemm_kernel, dim3(grid), dim3(kI4Threads), kI4SmemBytes, stream, 1,
+                    tm_a, tm_b, tm_sa, tm_sw, tm_l2, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -313,13 +351,21 @@ svdq_status quantize_act_impl(svdq_format format, int M, int K, int r, const voi
   p.xl1 = xl1;
   p.xl1_rest = r > 0 ? (static_rest ? d->xl1_scratch : xl1 + static_cast<size_t>(M) * r) : nullptr;
   p.status = d->status;
-  kern<<<dim3(ksplit, row_blocks, 1), kQaThreads, smem_bytes, static_cast<cudaStream_t>(stream)>>>(
-      tm_x, tm_l1, p);
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (launch_kernel(d, kern, dim3(ksplit, row_blocks, 1), dim3(kQaThreads), smem_bytes, cs, 1, tm_x,
+                    tm_l1, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
   if (r > 0 && ksplit > 1) {
     // xl1[0] += xl1[1] + ... + xl1[S-1], in order
     const size_t n4 = static_cast<size_t>(M) * r / 4;
-    xl1_reduce_kernel<<<grid_for(n4, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<float4*>(xl1), reinterpret_cast<const float4*>(p.xl1_rest), ksplit, n4);
+    if (launch_kernel(d, xl1_reduce_kernel, dim3(grid_for(n4, 256)), dim3(256), 0, cs, 1,
+                      reinterpret_cast<float4*>(xl1), reinterpret_cast<const float4*>(p.xl1_rest),
+                      ksplit, n4) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
   }
   return launch_status();
 }
@@ -451,23 +497,12 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.tiles = p.tiles_m * ((N + kGmBN - 1) / kGmBN);
   const int max_units = pair ? d->gemm_pairs : d->num_sms;
   const int units = p.tiles < max_units ? p.tiles : max_units;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(units * ctas, 1, 1);
-  cfg.blockDim = dim3(kGmThreads, 1, 1);
-  cfg.dynamicSmemBytes = pair ? GmCfg<true>::kSmemBytes : GmCfg<false>::kSmemBytes;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pair ? 1 : 0;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      pair ? cudaLaunchKernelEx(&cfg, w4a4_nvfp4_gemm_kernel<true>, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2,
-                                tm_y, p)
-           : cudaLaunchKernelEx(&cfg, w4a4_nvfp4_gemm_kernel<false>, tm_a, tm_b, tm_sfa, tm_sfb,
-                                tm_l2, tm_y, p);
+      pair ? launch_kernel(d, w4a4_nvfp4_gemm_kernel<true>, dim3(units * 2), dim3(kGmThreads),
+                           GmCfg<true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y, p)
+           : launch_kernel(d, w4a4_nvfp4_gemm_kernel<false>, dim3(units), dim3(kGmThreads),
+                           GmCfg<false>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y, p);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
@@ -526,10 +561,15 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
     p.Y = static_cast<__nv_bfloat16*>(Y) + static_cast<size_t>(m0) * N;
     p.status = d->status;
     const size_t smem = awq_smem_bytes(mm, K, kmb, stages);
-    if (kmb == 1)
-      awq_gemv_kernel<1><<<grid, kAwqThreads, smem, s>>>(tm_q, tm_sz, p);
-    else
-      awq_gemv_kernel<2><<<grid, kAwqThreads, smem, s>>>(tm_q, tm_sz, p);
+    const cudaError_t e =
+        kmb == 1 ? launch_kernel(d, awq_gemv_kernel<1>, dim3(grid), dim3(kAwqThreads), smem, s, 1,
+                                 tm_q, tm_sz, p)
+                 : launch_kernel(d, awq_gemv_kernel<2>, dim3(grid), dim3(kAwqThreads), smem, s, 1,
+                                 tm_q, tm_sz, p);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
   }
   return launch_status();
 }

@@ -150,6 +150,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   }
   tc_fence_before();
   if (kPair) cluster_sync(); else __syncthreads();  // barriers initialised in both CTAs
+  // everything above touches no global memory the previous grid may write
+  grid_dep_wait();
+  grid_dep_launch();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
