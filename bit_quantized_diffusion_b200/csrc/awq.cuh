@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
     }
     fence_barrier_init();
   }
-  __syncthreads();
+  cta_sync_converged();
   grid_dep_launch();
 
   if (warp == kAwqConsumers) {
@@ -340,6 +340,7 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
     const int m = p.M + i / G, g = i - (i / G) * G;
     xs[m * xs_ld + g] = 0.0f;
   }
+  __syncwarp();
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 
   // this lane's B-fragment runs: token rows r0 (+ 8 mb), lane quad t = lane % 4
@@ -395,6 +396,7 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
     for (int mb = 0; mb < kMB; ++mb)
       *reinterpret_cast<float4*>(red + ((warp * 32 + lane) * kMB + mb) * 4) =
           make_float4(acc[mb][0], acc[mb][1], acc[mb][2], acc[mb][3]);
+    __syncwarp();
     asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
     if (part == 0 && active && ok) {
 #pragma unroll
@@ -420,6 +422,7 @@ __global__ void __launch_bounds__(kAwqThreads, 1)
         }
       }
     }
+    __syncwarp();
     asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");  // red is free for the next round
   }
 }

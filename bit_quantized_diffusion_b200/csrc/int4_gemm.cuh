@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   grid_dep_wait();  // the prologue above touches no global memory the previous grid may write
   grid_dep_launch();
   tc_fence_after();
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -182,7 +182,7 @@ __global__ void debug_wait_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait(b, 0, status, limit_ns);
-  __syncthreads();
+  cta_sync_converged();
 }
 
 }  // namespace svdq

@@ -499,6 +499,20 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 
+// CTA / cluster barriers for code where a warp's lanes may have split (one
+// elected lane ran a producer or MMA loop, lanes left a wait loop at different
+// iterations): the barrier instructions are the warp-aligned forms, which
+// expect every lane of a warp to execute them together, so each warp
+// reconverges first.
+__device__ __forceinline__ void cta_sync_converged() {
+  __syncwarp();
+  __syncthreads();
+}
+__device__ __forceinline__ void cluster_sync_converged() {
+  __syncwarp();
+  cluster_sync();
+}
+
 __device__ __forceinline__ uint32_t map_peer_smem(uint32_t addr, uint32_t peer) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(peer));

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     }
   }
   tc_fence_before();
-  if (kPair) cluster_sync(); else __syncthreads();  // barriers initialised in both CTAs
+  if (kPair) cluster_sync_converged(); else cta_sync_converged();  // barriers initialised in both CTAs
   // everything above touches no global memory the previous grid may write
   grid_dep_wait();
   grid_dep_launch();
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   tc_fence_before();
   // both CTAs' tensor memory is written by the leader's MMAs: release it only
   // once every warp of the pair is done
-  if (kPair) cluster_sync(); else __syncthreads();
+  if (kPair) cluster_sync_converged(); else cta_sync_converged();
   if (warp == 1) {
     tc_fence_after();
     if (kPair) tmem_dealloc_pair(tmem, kTmCols);
