@@ -26,7 +26,7 @@
 //               16 (w % 8) .. + 15; lane l handles row 16 (w % 8) + l % 16 and
 //               columns 32 (l / 16) .. + 31 of the sub-chunk: two NVFP4 groups, or
 //               half an INT4 group (the other half is lane l ^ 16); the float32
-//               arithmetic runs on paired (f32x2) instructions
+//               arithmetic runs on paired (float2) instructions
 #pragma once
 
 #include "sm100.cuh"
@@ -203,120 +203,116 @@ __global__ void __launch_bounds__(kQaThreads, 1)
     const int half = lane >> 4;  // which 32 columns of the sub-chunk
     const int m = rb * 128 + row;
     const bool row_ok = m < p.M;
+    uint8_t* const code_row = p.codes + static_cast<size_t>(m) * (p.K / 2) + half * 16;
+    const uint32_t table_u32 = sbase + L.table;
     bool ok = true;
+    int s = 0;        // ring slot of stage i
+    uint32_t ph = 0;  // its phase parity
     for (int i = 0; i < nstage; ++i) {
-      const int s = i % NS;
-      ok = mbar_wait(bar_full(s), (i / NS) & 1, p.status);
+      const int slot = s;
+      ok = mbar_wait(bar_full(slot), ph, p.status);
       if (!ok) break;
+      if (++s == NS) {
+        s = 0;
+        ph ^= 1u;
+      }
       const int kc = kc0 + i * p.spc + sub;
       if (!active || kc >= kc1) {
         // nothing of this stage for this warp
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty(s));
+        if (lane == 0) mbar_arrive(bar_empty(slot));
         continue;
       }
-      const uint32_t sub_base = x_stage(s) + sub * L.sub_bytes;
-        // -- 32 bf16 of this row from the 128B-swizzled X tile, as float32 pairs
-        uint64_t xp[16];
-        {
-          const uint32_t rowbase = sub_base + row * 128;
-  #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int c = 4 * half + h;
-            uint32_t v0, v1, v2, v3;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
-                         : "r"(rowbase + ((c ^ (row & 7)) << 4)));
-            const uint32_t w[4] = {v0, v1, v2, v3};
-  #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              xp[4 * h + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
-          }
+      const uint32_t sub_base = x_stage(slot) + sub * L.sub_bytes;
+      // -- 32 bf16 of this row from the 128B-swizzled X tile, as 16 float pairs
+      float2 xv[16];
+      {
+        const uint32_t rowbase = sub_base + row * 128;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int c = 4 * half + h;
+          const uint4 v = lds_u4(rowbase + ((c ^ (row & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            xv[4 * h + j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
         }
-        // -- a1: smoothing, one float32 multiply per element
-        if (smoothing) {
-          const float4* sp = reinterpret_cast<const float4*>(smem + (sub_base - sbase) + L.sm_off) +
-                             8 * half;
-  #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 sv = sp[j];
-            xp[2 * j] = f2_mul(xp[2 * j], f2_pack(sv.x, sv.y));
-            xp[2 * j + 1] = f2_mul(xp[2 * j + 1], f2_pack(sv.z, sv.w));
-          }
+      }
+      // -- a1: smoothing, one float32 multiply per element
+      if (smoothing) {
+        const uint32_t sp = sub_base + L.sm_off + 128 * half;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 sv = lds_f4(sp + 16 * j);
+          xv[2 * j] = __fmul2_rn(xv[2 * j], make_float2(sv.x, sv.y));
+          xv[2 * j + 1] = __fmul2_rn(xv[2 * j + 1], make_float2(sv.z, sv.w));
         }
-        // this warp no longer reads the stage's shared memory
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty(s));
-        // -- a2 + a3: group scale and codes
-        float xh[32];
-  #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float2 v = f2_unpack(xp[j]);
-          xh[2 * j] = v.x;
-          xh[2 * j + 1] = v.y;
-        }
-        uint32_t code[4];
-        if (kFmt == 0) {
-          uint32_t sc[2];
-  #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            float amax = 0.0f;
-  #pragma unroll
-            for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xh[16 * g + j]));
-            sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
-            const float2 vr = table[sc[g]];  // (decoded scale, its reciprocal)
-            const uint64_t rcp2 = f2_pack(vr.y, vr.y);
-            float y0[8], y1[8];
-  #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 a = f2_unpack(f2_mul(xp[8 * g + j], rcp2));
-              const float2 b = f2_unpack(f2_mul(xp[8 * g + 4 + j], rcp2));
-              y0[2 * j] = a.x;
-              y0[2 * j + 1] = a.y;
-              y1[2 * j] = b.x;
-              y1[2 * j + 1] = b.y;
-            }
-            const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
-            code[2 * g] = live ? e2m1x8(y0) : 0u;
-            code[2 * g + 1] = live ? e2m1x8(y1) : 0u;
-          }
-          // the row's four scale bytes: groups 2 half, 2 half + 1 here, the others in lane ^ 16
-          const uint32_t mine = sc[0] | (sc[1] << 8);
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
-          if (half == 0) {
-            const uint32_t word = mine | (other << 16);
-            const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
-            *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
-                word;
-          }
-        } else {
+      }
+      // this warp no longer reads the stage's shared memory
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(slot));
+      // -- a2 + a3: group scale and codes
+      uint32_t code[4];
+      if (kFmt == 0) {
+        uint32_t sc[2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
           float amax = 0.0f;
-  #pragma unroll
-          for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xh[j]));
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-          const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
-          const float sval = __half2float(hs);
-  #pragma unroll
-          for (int w = 0; w < 4; ++w) code[w] = 0u;
-          if (sval != 0.0f) {
-            const float rcp = __frcp_rn(sval);
-  #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              int v = __float2int_rn(__fmul_rn(xh[j], rcp));
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            amax = fmaxf(amax, fmaxf(fabsf(xv[8 * g + j].x), fabsf(xv[8 * g + j].y)));
+          sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
+          const float2 vr = lds_f2(table_u32 + 8 * sc[g]);  // (decoded scale, its reciprocal)
+          const float2 rcp2 = make_float2(vr.y, vr.y);
+          float2 y0[4], y1[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            y0[j] = __fmul2_rn(xv[8 * g + j], rcp2);
+            y1[j] = __fmul2_rn(xv[8 * g + 4 + j], rcp2);
+          }
+          const bool live = vr.x != 0.0f;  // a zero scale stores zero codes
+          code[2 * g] = live ? e2m1x8(y0) : 0u;
+          code[2 * g + 1] = live ? e2m1x8(y1) : 0u;
+        }
+        // the row's four scale bytes: groups 2 half, 2 half + 1 here, the others in lane ^ 16
+        const uint32_t mine = sc[0] | (sc[1] << 8);
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
+        if (half == 0) {
+          const uint32_t word = mine | (other << 16);
+          const size_t atom = static_cast<size_t>(rb) * kc_total + kc;
+          *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) = word;
+        }
+      } else {
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(xv[j].x), fabsf(xv[j].y)));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+        const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        const float sval = __half2float(hs);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) code[w] = 0u;
+        if (sval != 0.0f) {
+          const float rcp = __frcp_rn(sval);
+          const float2 rcp2 = make_float2(rcp, rcp);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float2 q = __fmul2_rn(xv[j], rcp2);
+            const float qq[2] = {q.x, q.y};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              int v = __float2int_rn(qq[e]);
               v = max(-7, min(7, v));
               // tiled INT4 codes are sign-magnitude nibbles
               const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
-              code[j >> 3] |= nib << (4 * (j & 7));
+              code[j >> 2] |= nib << (4 * (2 * (j & 3) + e));
             }
           }
-          if (half == 0)
-            reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] =
-                hs;
         }
-        if (row_ok) {
-          *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) + kc * 32 + half * 16) =
-              make_uint4(code[0], code[1], code[2], code[3]);
-        }
+        if (half == 0)
+          reinterpret_cast<__half*>(p.scales)[static_cast<size_t>(kc) * p.m_pad + rb * 128 + row] = hs;
+      }
+      if (row_ok)
+        *reinterpret_cast<uint4*>(code_row + kc * 32) = make_uint4(code[0], code[1], code[2], code[3]);
     }
     // ------------------------------------------------------------ xl1 epilogue
     // this split's partial down-projection of the CTA's 128 rows

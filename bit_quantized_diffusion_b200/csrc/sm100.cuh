@@ -519,6 +519,28 @@ __device__ __forceinline__ uint32_t map_peer_smem(uint32_t addr, uint32_t peer) 
   return r;
 }
 
+// Shared-memory loads by address. Volatile, so they stay behind the barrier
+// waits (also volatile asm) that publish the data.
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -533,7 +555,7 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 // packed into 32 bits: element i in bits 4i..4i+3.
 __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
@@ -545,10 +567,25 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
   return out;
 }
 
+// The same for four float pairs: pair k holds elements 2k (x) and 2k + 1 (y).
+__device__ __forceinline__ uint32_t e2m1x8(const float2 (&v)[4]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x),
+        "f"(v[3].y));
+  return out;
+}
+
 // float32 >= 0 -> E4M3 code (round-to-nearest-even, saturate to 448).
 __device__ __forceinline__ uint32_t e4m3_code(float v) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
   return out & 0xFFu;
 }
 
