@@ -59,25 +59,6 @@ __global__ void unpack_int4_scales_kernel(const uint16_t* tiled, uint16_t* plain
   }
 }
 
-// INT4 codes: plain two's-complement nibbles <-> tiled sign-magnitude nibbles
-// (values -7..7; the nibble order of the bytes is unchanged).
-__device__ __forceinline__ uint32_t int4_nibble_to_sm(uint32_t n) {
-  return n >= 8u ? 8u | (16u - n) : n;
-}
-__device__ __forceinline__ uint32_t int4_nibble_from_sm(uint32_t n) {
-  return n >= 8u ? (16u - (n & 7u)) & 15u : n;
-}
-
-__global__ void int4_codes_kernel(const uint8_t* src, uint8_t* dst, size_t n, int to_tiled) {
-  for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n;
-       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint32_t b = src[t];
-    const uint32_t lo = b & 15u, hi = b >> 4;
-    dst[t] = static_cast<uint8_t>(to_tiled ? int4_nibble_to_sm(lo) | (int4_nibble_to_sm(hi) << 4)
-                                           : int4_nibble_from_sm(lo) | (int4_nibble_from_sm(hi) << 4));
-  }
-}
-
 __global__ void copy_bytes_kernel(const uint4* src, uint4* dst, size_t n16) {
   for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n16;
        t += static_cast<size_t>(gridDim.x) * blockDim.x)

@@ -302,8 +302,7 @@ __global__ void __launch_bounds__(kQaThreads, 1)
             for (int e = 0; e < 2; ++e) {
               int v = __float2int_rn(qq[e]);
               v = max(-7, min(7, v));
-              // tiled INT4 codes are sign-magnitude nibbles
-              const uint32_t nib = v < 0 ? 8u | static_cast<uint32_t>(-v) : static_cast<uint32_t>(v);
+              const uint32_t nib = static_cast<uint32_t>(v) & 15u;  // two's complement nibble
               code[j >> 2] |= nib << (4 * (2 * (j & 3) + e));
             }
           }

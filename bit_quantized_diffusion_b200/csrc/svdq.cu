@@ -36,7 +36,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
-  int gemm_pairs = 0;  // co-resident clusters of the CTA-pair GEMM
+  int gemm_pairs = 0;  // co-resident clusters of the CTA-pair NVFP4 GEMM
+  int int4_pairs = 0;  // the same for the INT4 GEMM
   int gemm_pair_mode = -1;  // -1: by shape; SVDQ_GEMM_PAIR=0/1 forces single-CTA / CTA-pair tiles
   uint32_t* status = nullptr;
   float* xl1_scratch = nullptr;  // device address of g_xl1_scratch
@@ -119,7 +120,9 @@ svdq_status device_setup(DeviceInfo** out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(GmCfg<true>::kSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
-    if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_int4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kI4SmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     // all of the SM's unified L1/shared storage as shared memory, so that the
@@ -128,7 +131,8 @@ svdq_status device_setup(DeviceInfo** out) {
                           reinterpret_cast<const void*>(quantize_act_kernel<1>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<false>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true>),
-                          reinterpret_cast<const void*>(w4a4_int4_gemm_kernel),
+                          reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<false>),
+                          reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<true>),
                           reinterpret_cast<const void*>(awq_gemv_kernel<1>),
                           reinterpret_cast<const void*>(awq_gemv_kernel<2>)})
       if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -142,28 +146,30 @@ svdq_status device_setup(DeviceInfo** out) {
     {
       // how many 2-CTA clusters of the pair GEMM can be resident at once (a
       // persistent grid larger than that would run its last clusters late)
-      cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * (d.num_sms / 2), 1, 1);
-      q.blockDim = dim3(kGmThreads, 1, 1);
-      q.dynamicSmemBytes = GmCfg<true>::kSmemBytes;
-      cudaLaunchAttribute a[1];
-      a[0].id = cudaLaunchAttributeClusterDimension;
-      a[0].val.clusterDim.x = 2;
-      a[0].val.clusterDim.y = 1;
-      a[0].val.clusterDim.z = 1;
-      q.attrs = a;
-      q.numAttrs = 1;
-      int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, w4a4_nvfp4_gemm_kernel<true>, &q) !=
-              cudaSuccess ||
-          clusters <= 0) {
-        (void)cudaGetLastError();
-        clusters = d.num_sms / 2;
-      }
-      d.gemm_pairs = clusters < d.num_sms / 2 ? clusters : d.num_sms / 2;
+      auto pairs = [&](auto kern, int threads, size_t smem) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(2 * (d.num_sms / 2), 1, 1);
+        q.blockDim = dim3(threads, 1, 1);
+        q.dynamicSmemBytes = smem;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = 2;
+        a[0].val.clusterDim.y = 1;
+        a[0].val.clusterDim.z = 1;
+        q.attrs = a;
+        q.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &q) != cudaSuccess || clusters <= 0) {
+          (void)cudaGetLastError();
+          clusters = d.num_sms / 2;
+        }
+        return clusters < d.num_sms / 2 ? clusters : d.num_sms / 2;
+      };
+      d.gemm_pairs = pairs(w4a4_nvfp4_gemm_kernel<true>, kGmThreads, GmCfg<true>::kSmemBytes);
+      d.int4_pairs = pairs(w4a4_int4_gemm_kernel<true>, kI4Threads, kI4SmemBytes);
       if (std::getenv("SVDQ_DEBUG") != nullptr)
-        std::fprintf(stderr, "svdq: %d SMs, %d co-resident GEMM CTA pairs\n", d.num_sms,
-                     d.gemm_pairs);
+        std::fprintf(stderr, "svdq: %d SMs, %d / %d co-resident NVFP4 / INT4 GEMM CTA pairs\n",
+                     d.num_sms, d.gemm_pairs, d.int4_pairs);
     }
     if (const char* e = std::getenv("SVDQ_GEMM_PAIR")) d.gemm_pair_mode = std::atoi(e) != 0;
     if (const char* e = std::getenv("SVDQ_PDL")) d.pdl = std::atoi(e) != 0;
@@ -232,22 +238,26 @@ unsigned grid_for(size_t n, unsigned threads) {
   return static_cast<unsigned>(b);
 }
 
-// INT4 W4A4 GEMM (w4a4_int4_gemm_kernel): packed codes [rows, K/2] as 64-byte
-// boxes, group-major FP16 scales [K/64][rows padded to 128] as 2-group boxes.
+// INT4 W4A4 GEMM (w4a4_int4_gemm_kernel): packed codes [rows, K/2] as one-group
+// boxes [128 rows x 32 B], group-major FP16 scales [K/64][rows padded to 128]
+// as one-group boxes [128], Y as 32 x 32 TMA-store boxes. CTA pairs whenever M
+// exceeds one 128-row block, as for NVFP4.
 svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
                              const void* w_scales, const void* L2, const void* bias, void* Y,
                              int ldy, svdq_out out, cudaStream_t stream) {
-  CUtensorMap tm_a, tm_b, tm_sa, tm_sw, tm_l2;
+  const bool pair = (d->gemm_pair_mode < 0 ? true : d->gemm_pair_mode != 0) && M > kI4BM;
+  const int ctas = pair ? 2 : 1;
+  CUtensorMap tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y;
   const uint64_t G = static_cast<uint64_t>(K / 64);
-  if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 64, kI4BM,
+  if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 32, kI4BM,
                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 64, kI4BN,
+      !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 32, kI4BM,
                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_2d(&tm_sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_scales, pad128(M), G, pad128(M) * 2,
-                    128, 2, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                    128, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_tmap_2d(&tm_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w_scales, pad128(N), G, pad128(N) * 2,
-                    128, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    128, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, N, r,
@@ -256,6 +266,13 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
   } else {
     tm_l2 = tm_a;
   }
+  // output: 32 x 32 boxes, bf16 rows of 64 B (64-byte swizzle) or f32 rows of 128 B
+  const bool f32 = out == SVDQ_OUT_F32;
+  const int esz = f32 ? 4 : 2;
+  if (!make_tmap_2d(&tm_y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    Y, N, M, static_cast<uint64_t>(ldy) * esz, 32, 32,
+                    f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    return SVDQ_ERR_CUDA;
   I4Params p;
   p.M = M;
   p.N = N;
@@ -263,15 +280,18 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
   p.r = r;
   p.xl1 = xl1;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
-  p.Y = Y;
-  p.ldy = ldy;
-  p.out_f32 = out == SVDQ_OUT_F32;
+  p.out_f32 = f32;
   p.status = d->status;
-  p.tiles_m = (M + kI4BM - 1) / kI4BM;
+  p.tiles_m = (M + kI4BM * ctas - 1) / (kI4BM * ctas);
   p.tiles = p.tiles_m * ((N + kI4BN - 1) / kI4BN);
-  const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
-  if (launch_kernel(d, w4a4_int4_gemm_kernel, dim3(grid), dim3(kI4Threads), kI4SmemBytes, stream, 1,
-                    tm_a, tm_b, tm_sa, tm_sw, tm_l2, p) != cudaSuccess) {
+  const int max_units = pair ? d->int4_pairs : d->num_sms;
+  const int units = p.tiles < max_units ? p.tiles : max_units;
+  const cudaError_t e =
+      pair ? launch_kernel(d, w4a4_int4_gemm_kernel<true>, dim3(units * 2), dim3(kI4Threads),
+                           kI4SmemBytes, stream, 2, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p)
+           : launch_kernel(d, w4a4_int4_gemm_kernel<false>, dim3(units), dim3(kI4Threads),
+                           kI4SmemBytes, stream, 1, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p);
+  if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }
@@ -597,12 +617,9 @@ svdq_status svdq_pack(svdq_pack_kind kind, svdq_format format, int rows, int K,
     if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
     if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
     const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
-    if (format == SVDQ_NVFP4_G16)
-      copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(plain_codes),
-                                                       static_cast<uint4*>(tiled_codes), n16);
-    else
-      int4_codes_kernel<<<grid_for(n16 * 16, T), T, 0, s>>>(
-          static_cast<const uint8_t*>(plain_codes), static_cast<uint8_t*>(tiled_codes), n16 * 16, 1);
+    // the tiled codes of both formats are the plain bytes
+    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(plain_codes),
+                                                     static_cast<uint4*>(tiled_codes), n16);
     if (format == SVDQ_NVFP4_G16) {
       const size_t n = pad128(rows) * (K / 16);
       pack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(
@@ -653,12 +670,8 @@ svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K
     if (plain_zeros != nullptr) return SVDQ_ERR_INVALID_ARG;
     if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
     const size_t n16 = static_cast<size_t>(rows) * (K / 2) / 16;
-    if (format == SVDQ_NVFP4_G16)
-      copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(tiled_codes),
-                                                       static_cast<uint4*>(plain_codes), n16);
-    else
-      int4_codes_kernel<<<grid_for(n16 * 16, T), T, 0, s>>>(
-          static_cast<const uint8_t*>(tiled_codes), static_cast<uint8_t*>(plain_codes), n16 * 16, 0);
+    copy_bytes_kernel<<<grid_for(n16, T), T, 0, s>>>(static_cast<const uint4*>(tiled_codes),
+                                                     static_cast<uint4*>(plain_codes), n16);
     if (format == SVDQ_NVFP4_G16) {
       const size_t n = static_cast<size_t>(rows) * (K / 16);
       unpack_nvfp4_scales_kernel<<<grid_for(n, T), T, 0, s>>>(

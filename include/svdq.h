@@ -68,11 +68,9 @@ int svdq_version(void);
 /*
  * Buffer sizes in bytes of the storage formats below. Codes are row-major
  * packed nibbles, K contiguous, element 2j in the low nibble, 2j+1 in the high
- * nibble: rows * K / 2 bytes. NVFP4 codes are E2M1 in both the plain and the
- * tiled form. INT4 values (-7..7) are two's-complement nibbles in the plain
- * form and sign-magnitude nibbles (8 + |v| for v < 0) in the tiled form, which
- * the GEMM expands to 8-bit tensor-core operands with three logic operations
- * per four codes.
+ * nibble: rows * K / 2 bytes. NVFP4 codes are E2M1 and INT4 values (-7..7) are
+ * two's complement nibbles, in both the plain and the tiled form (the same
+ * bytes).
  * Scales ("tiled"):
  *  - NVFP4: rows padded to 128; for row m and scale column j = k/16 the byte sits
  *    in 512-byte atom a = (m/128) * (K/64) + j/4 at offset
@@ -170,9 +168,11 @@ svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, c
  * Y                  device, [M, ldy] bf16 (out = SVDQ_OUT_BF16) or float32, ldy >= N,
  *                    ldy * element size % 16 == 0
  * The low-rank product uses xl1 split into two bf16 terms; accumulation is float32.
- * NVFP4 runs on the block-scaled FP4 MMA. INT4 has no integer 4-bit MMA on
- * sm_100a: each 64-wide group's product is formed exactly on the tensor cores
- * (codes as E4M3 values v/512) and scaled by s_a s_w on the CUDA cores.
+ * NVFP4 runs on the block-scaled FP4 MMA. INT4 has no 4-bit integer MMA on
+ * sm_100a: both operands are dequantized on chip to FP16 values fp16(s q) (one
+ * rounding, relative error <= 2^-12; exact for power-of-two scales) and
+ * multiplied on the FP16 tensor cores with float32 accumulation. |s q| must fit
+ * FP16 (group absolute maxima below 65504).
  */
 svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
@@ -202,9 +202,8 @@ svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, cons
  * svdq_pack / svdq_unpack -- convert between plain and tiled storage
  * (unpack(pack(x)) == x bit for bit).
  *
- * ACT / WEIGHT: plain_codes [rows, K/2] bytes -> tiled codes (NVFP4: the same
- *   bytes; INT4: two's complement -> sign-magnitude per nibble, where -8 is out
- *   of contract);
+ * ACT / WEIGHT: plain_codes [rows, K/2] bytes -> tiled codes (the same bytes,
+ *   NVFP4 and INT4);
  *   plain_scales: NVFP4 uint8 [rows, K/16] E4M3 codes, INT4 fp16 [rows, K/64]
  *   -> tiled scales (layouts above). plain_zeros must be NULL.
  * AWQ: plain_codes = qweight [N, K/2] (element 2j low nibble, values 0..15),

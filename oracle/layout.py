@@ -18,9 +18,8 @@ INT4 scales (activations and weights), group-major
 
 NVFP4 / INT4 codes
     Plain: row-major, K contiguous, two codes per byte, element 2j in the low
-    nibble (INT4 as two's complement). The tiled NVFP4 codes are the same bytes.
-    Tiled INT4 codes hold each value v in -7..7 as a sign-magnitude nibble:
-    8 + |v| if v < 0, else v; nibble order as in the plain form.
+    nibble (INT4 as two's complement). The tiled codes of both formats are the
+    same bytes (INT4 values -7..7 as two's complement nibbles, v & 15).
 
 AWQ qweight, MMA-fragment order
     N padded to 16 rows. For row block b = n // 16 and group g = k // 64 there
@@ -96,11 +95,11 @@ def untile_int4_scales(tiled: np.ndarray, rows: int, K: int) -> np.ndarray:
 
 # --------------------------------------------------------------- INT4 codes
 def tile_int4_codes(q: np.ndarray) -> np.ndarray:
-    """q [rows, K] integers in -7..7 -> tiled bytes [rows, K/2] (sign-magnitude nibbles)."""
+    """q [rows, K] integers in -7..7 -> tiled bytes [rows, K/2] (two's complement nibbles)."""
     q = np.asarray(q).astype(np.int16)
     if np.any(np.abs(q) > 7):
         raise ValueError("INT4 codes must lie in -7..7")
-    nib = np.where(q < 0, 8 - q, q).astype(np.uint8)  # 8 + |q| for negative q
+    nib = (q & 0xF).astype(np.uint8)  # v & 15
     return (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
 
 
@@ -110,7 +109,7 @@ def untile_int4_codes(tiled: np.ndarray) -> np.ndarray:
     nib = np.empty(t.shape[:-1] + (t.shape[-1] * 2,), dtype=np.int16)
     nib[..., 0::2] = t & 0xF
     nib[..., 1::2] = t >> 4
-    return np.where(nib >= 8, -(nib - 8), nib).astype(np.int16)
+    return np.where(nib >= 8, nib - 16, nib).astype(np.int16)
 
 
 # --------------------------------------------------------------- AWQ qweight

@@ -46,7 +46,7 @@ def oracle_layer(shape: WL.SvdqShape, M: int | None = None) -> dict:
 
 
 def tiled_codes(fmt: str, q: np.ndarray) -> np.ndarray:
-    """Codes as the kernels store them: NVFP4 plain packed nibbles, INT4 sign-magnitude."""
+    """Codes as the kernels store them: packed nibbles (INT4 two's complement)."""
     if fmt == "nvfp4":
         return S.pack_nibbles(q).reshape(-1)
     return LO.tile_int4_codes(q).reshape(-1)

@@ -142,7 +142,13 @@ def test_w4a4_linear_matches_oracle(bq, shape, with_bias):
     assert bq.svdq_check_device_status() == 0
     y32 = y32.cpu().numpy().astype(np.float64)
     y16 = y16.float().cpu().numpy().astype(np.float64)
-    assert C.rel_l2(y32, ref) <= 1e-5, f"float32 output rel-L2 {C.rel_l2(y32, ref):.3e}"
+    # NVFP4 operands are exact on the tensor cores: only float32 accumulation
+    # order separates the result from the oracle. INT4 operands are dequantized
+    # to FP16 first, one rounding each (at most 2^-12 relative), so a product is
+    # within 2^-11 relative; the bound is that, four times inside the stated
+    # output tolerance (relative L2 <= 2e-3).
+    bound = 1e-5 if fmt == "nvfp4" else 2.0 ** -11
+    assert C.rel_l2(y32, ref) <= bound, f"float32 output rel-L2 {C.rel_l2(y32, ref):.3e}"
     C.assert_gemm_close(y32, ref, bf16_out=False, what="Y f32")
     C.assert_gemm_close(y16, ref, bf16_out=True, what="Y bf16")
 
@@ -234,7 +240,7 @@ def test_pack_unpack_round_trip(bq, fmt):
     else:
         q = rng.integers(-7, 8, size=(rows, K))
         codes = S.pack_nibbles(q).reshape(-1)          # plain: two's complement
-        want_codes = C.tiled_codes("int4", q)          # tiled: sign-magnitude
+        want_codes = C.tiled_codes("int4", q)          # tiled: the same bytes
     if fmt == "nvfp4":
         plain = rng.integers(0, 127, size=(rows, K // 16)).astype(np.uint8)
         want = LO.tile_nvfp4_scales(plain)

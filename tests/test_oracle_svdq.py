@@ -141,12 +141,13 @@ def test_nvfp4_scale_atom_positions():
 
 
 def test_int4_code_tiling_hand_bytes():
-    # values (element 2j low nibble): (1, -1) -> 0x91, (-7, 7) -> 0x7F, (0, -3) -> 0xB0
+    # values (element 2j low nibble), two's complement: (1, -1) -> 0xF1,
+    # (-7, 7) -> 0x79, (0, -3) -> 0xD0
     q = np.array([[1, -1, -7, 7, 0, -3]])
     t = L.tile_int4_codes(q)
-    assert t.tolist() == [[0x91, 0x7F, 0xB0]]
+    assert t.tolist() == [[0xF1, 0x79, 0xD0]]
     assert np.array_equal(L.untile_int4_codes(t), q)
-    # the plain form of the same values is two's complement
+    # the plain form holds the same bytes
     assert S.pack_nibbles(q).tolist() == [[0xF1, 0x79, 0xD0]]
     every = np.arange(-7, 8).repeat(2).reshape(1, -1)
     assert np.array_equal(L.untile_int4_codes(L.tile_int4_codes(every)), every)
