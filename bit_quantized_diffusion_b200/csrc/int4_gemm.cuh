@@ -27,25 +27,26 @@
 // Two disjoint 256-column accumulators (no scale factors live in tensor
 // memory) let the next tile's MMAs run while the epilogue drains the last one.
 //
-// Warp roles per CTA (18 warps):
+// Warp roles per CTA (22 warps):
 //   warp 0      TMA producer: packed A and B codes [128 rows x 32 B] and their
 //               FP16 scales [128] for one group per packed-ring stage
 //   warp 1      tensor-memory owner; in the leader CTA also the MMA issuer
-//   warps 2-9   converters: packed ring -> FP16 operand ring (128-byte swizzle,
-//               one row per thread); for a low-rank slot, the L2 chunk by TMA
-//               and xl1 as bf16 hi + lo operand tiles
-//   warps 10-17 epilogue, two warps per tensor-memory lane quadrant:
-//               accumulator -> + bias -> bf16 / f32 -> swizzled shared memory ->
-//               TMA store
+//   warps 2-17  converters: packed ring -> FP16 operand ring (128-byte swizzle,
+//               half a row per thread: the dequantization's dependent steps need
+//               many warps to hide them); for a low-rank slot, the L2 chunk by
+//               TMA and xl1 as bf16 hi + lo operand tiles
+//   warps 18-21 epilogue, one warp per tensor-memory lane quadrant (it is idle
+//               for most of a tile): accumulator -> + bias -> bf16 / f32 ->
+//               swizzled shared memory -> TMA store
 #pragma once
 
 #include "sm100.cuh"
 
 namespace svdq {
 
-constexpr int kI4Threads = 576;
-constexpr int kI4CvtWarps = 8;
-constexpr int kI4EpiWarps = 8;
+constexpr int kI4Threads = 704;
+constexpr int kI4CvtWarps = 16;
+constexpr int kI4EpiWarps = 4;
 constexpr int kI4BM = 128, kI4BN = 256;               // rows per CTA, columns per tile
 constexpr int kI4PkOp = 128 * 32;                     // one operand's packed codes, one group
 constexpr int kI4PkStage = 2 * kI4PkOp + 2 * 128 * 2; // A, B codes; A, B FP16 scales: 8.5 KB
@@ -58,9 +59,9 @@ constexpr int kI4LrATile = 128 * kI4LrK * 2;          // 8 KB per bf16 tile (hi,
 constexpr int kI4StageOut = 4096;                     // epilogue staging bytes per warp
 constexpr uint32_t kI4OffOp = 0;
 constexpr uint32_t kI4OffPk = kI4OffOp + kI4OpStages * kI4OpStage;
-constexpr uint32_t kI4OffOut = kI4OffPk + kI4PkStages * kI4PkStage;
+constexpr uint32_t kI4OffOut = (kI4OffPk + kI4PkStages * kI4PkStage + 1023) / 1024 * 1024;
 constexpr uint32_t kI4OffBias = kI4OffOut + kI4EpiWarps * kI4StageOut;
-constexpr uint32_t kI4OffBars = kI4OffBias + kI4EpiWarps * 128 * 4;
+constexpr uint32_t kI4OffBars = kI4OffBias + kI4EpiWarps * 256 * 4;
 constexpr int kI4NumBars = 2 * kI4PkStages + 2 * kI4OpStages + 4;
 constexpr uint32_t kI4OffTmemSlot = kI4OffBars + 8 * kI4NumBars;
 constexpr size_t kI4SmemBytes = kI4OffTmemSlot + 16 + 1024;  // + alignment slack
@@ -108,8 +109,10 @@ __device__ __forceinline__ void int4x8_dequant(uint32_t w, __half2 s2, uint32_t 
   }
 }
 
+// 22 warps: up to six share one of the SM's four 16K-register partitions, which
+// caps the kernel at 80 registers per thread.
 template <bool kPair>
-__global__ void __launch_bounds__(kI4Threads, 1)
+__global__ void __maxnreg__(80)
     w4a4_int4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_sa,
@@ -272,9 +275,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
   } else if (warp < 2 + kI4CvtWarps) {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - 64;           // 0..255
-    const int op = ct >> 7;                    // 0: an A row, 1: a B row
+    const int ct = threadIdx.x - 64;           // 0..511
+    const int op = (ct >> 7) & 1;              // 0: an A row, 1: a B row
     const int row = ct & 127;
+    const int hk = ct >> 8;                    // which 32 of the row's 64 K
     bool ok = true;
     int jp = 0, jo = 0;
     for (int i = 0; i < my_tiles && ok; ++i) {
@@ -290,20 +294,21 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           ok = mbar_wait(pk_full(ps), (jp / NP) & 1, p.status) &&
                mbar_wait(op_empty(s), ((jo / NO) & 1) ^ 1, p.status);
           if (!ok) break;
-          const uint32_t src = pk_st(ps) + op * kI4PkOp + row * 32;
-          const uint4 c0 = lds_u4(src), c1 = lds_u4(src + 16);
+          const uint32_t src = pk_st(ps) + op * kI4PkOp + row * 32 + hk * 16;
+          const uint4 c0 = lds_u4(src);
           uint16_t sc;
           asm volatile("ld.shared.u16 %0, [%1];"
                        : "=h"(sc)
                        : "r"(pk_st(ps) + 2 * kI4PkOp + op * 256 + row * 2));
           const __half2 s2 = __halves2half2(__ushort_as_half(sc), __ushort_as_half(sc));
-          // this thread's 64 FP16 values: 16-byte chunk c = codes 8c .. 8c + 7
+          // this thread's 32 FP16 values: 16-byte chunk c = codes 8c .. 8c + 7
           const uint32_t rowp = st + op * kI4OpTile + row * 128;
-          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = 4 * hk + cc;
             uint32_t o[4];
-            int4x8_dequant(w[c], s2, o);
+            int4x8_dequant(w[cc], s2, o);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                              rowp + ((c ^ (row & 7)) << 4)),
                          "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
@@ -325,7 +330,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           // so the global read overlaps it); one thread brings this CTA's L2 chunk
           const int c = kt - G;
           float v[kI4LrK];
-          if (op == 0) {
+          const bool stager = op == 0 && hk == 0;  // one thread per A row
+          if (stager) {
             const float4* srcx =
                 reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r + c * kI4LrK);
 #pragma unroll
@@ -351,7 +357,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                 tma_load_2d(st + nb * (kI4LrK * 128), &tm_l2, fb, nrow + nb * 64, c * kI4LrK);
             }
           }
-          if (op == 0) {
+          if (stager) {
             const uint32_t a_hi = st + kI4OpTile, a_lo = a_hi + kI4LrATile;
 #pragma unroll
             for (int cm = 0; cm < kI4LrK / 8; ++cm) {
@@ -385,13 +391,11 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Each warp owns four 32-column sub-tiles of its lane quadrant: columns
-    // 128 half .. 128 half + 127 of the 256.
-    const int ew = warp - 2 - kI4CvtWarps;   // 0..7
+    // Each warp owns the eight 32-column sub-tiles of its lane quadrant.
+    const int ew = warp - 2 - kI4CvtWarps;   // 0..3
     const int quad = warp & 3;               // tensor-memory lanes 32 quad .. 32 quad + 31
-    const int half = ew >> 2;
     const uint32_t out_buf = sbase + kI4OffOut + ew * kI4StageOut;
-    float* bias_s = reinterpret_cast<float*>(smem + kI4OffBias) + ew * 128;  // [4][32]
+    float* bias_s = reinterpret_cast<float*>(smem + kI4OffBias) + ew * 256;  // [8][32]
     bool ok = true;
     int stores = 0;
     for (int i = 0; i < my_tiles && ok; ++i) {
@@ -403,20 +407,20 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       // bias for this warp's sub-tiles, fetched before the accumulator is ready
       __syncwarp();
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int n = n0 + 128 * half + 32 * t + lane;
+      for (int t = 0; t < 8; ++t) {
+        const int n = n0 + 32 * t + lane;
         bias_s[t * 32 + lane] = (p.bias != nullptr && n < p.N) ? __bfloat162float(p.bias[n]) : 0.0f;
       }
       __syncwarp();
       ok = mbar_wait(acc_full(b), u & 1, p.status);
       if (!ok) break;
       tc_fence_after();
-      for (int t = 0; t < 4; ++t) {
-        const int j0 = 128 * half + 32 * t;
+      for (int t = 0; t < 8; ++t) {
+        const int j0 = 32 * t;
         uint32_t acc[32];
         tmem_ld32(t_row + j0, acc);
         tmem_ld_wait();
-        if (t == 3) {
+        if (t == 7) {
           // the warp's whole slice is in registers: the accumulator is free
           tc_fence_before();
           __syncwarp();
