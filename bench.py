@@ -10,8 +10,10 @@ One step is one pass of the whole hot path over one batch of synthetic input:
                            (M = 4, K = 3072, N = 18432)
 The metric is TFLOP/s over the step: 2MNK + 2Mr(K+N) for the SVDQ layer plus
 2MNK for the AWQ layer, divided by the device time of the step. L2 is flushed
-(a 256 MiB write) before every step, outside the timed events. The kernels of
-a step are launched with programmatic dependent launch, so each one's launch
+before every step, outside the timed events: a 256 MiB write, then a 256 MiB
+read, so the step starts with none of its inputs in L2 and with no dirty lines
+left from the flush (their write-back would otherwise land inside the step).
+The kernels of a step are launched with programmatic dependent launch, so each one's launch
 and prologue overlap the previous kernel's tail; the timed region therefore
 records events only at step boundaries, and the per-kernel times (and the
 roofline of the GEMM) come from a second pass of the same steps with an event
@@ -313,7 +315,8 @@ def config_block(n_gpus: int) -> dict:
                         f"r={SHAPE.r} NVFP4 g16 + bias; AWQ W4A16 M={AWQ.M} K={AWQ.K} N={AWQ.N} g64",
             "M": SHAPE.M, "K": SHAPE.K, "N": SHAPE.N, "r": SHAPE.r, "format": "nvfp4_g16",
             "awq": {"M": AWQ.M, "K": AWQ.K, "N": AWQ.N, "group": AWQ.group},
-            "l2": "flushed before every step (256 MiB write, outside the timed events)",
+            "l2": "flushed before every step: 256 MiB write, then 256 MiB read (clean lines), "
+                  "outside the timed events",
             "parallelism": f"dp{n_gpus} (independent token batches per GPU, no collective)"}
 
 
@@ -370,7 +373,14 @@ def main() -> None:
     xl1 = torch.empty((bq.svdq_xl1_splits(M, K, r), M, r), dtype=torch.float32, device=dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     Ya = torch.empty((AWQ.M, AWQ.N), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush():
+        # evict the step's inputs, then replace the dirty lines the write left
+        # in L2 with clean ones
+        flush_w.zero_()
+        flush_r.sum()
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -385,7 +395,7 @@ def main() -> None:
         bq.awq_w4a16_linear(Xa, awq_w["qweight"], awq_w["sz"], bias_a, AWQ.N, Y=Ya, stream=stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     if bq.svdq_check_device_status() != 0:
@@ -405,7 +415,7 @@ def main() -> None:
         # event recorded between two kernels keeps the second from being
         # launched while the first finishes)
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             ev_s[i].record(stream)
             step()
             ev_e[i].record(stream)
@@ -415,7 +425,7 @@ def main() -> None:
         # the kernel-timing pass: the same K steps with an event between every
         # two kernels; each kernel's time here includes its launch gap
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             ev_ks[i].record(stream)
             step(ev_k[i])
             ev_ke[i].record(stream)
@@ -446,7 +456,7 @@ def main() -> None:
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(e2e_steps):
-        flush.zero_()
+        flush()
         e_s[i].record(stream)
         X.copy_(Xh, non_blocking=True)
         Xa.copy_(Xah, non_blocking=True)

@@ -88,6 +88,39 @@ __host__ inline size_t qa_smem_bytes(int r, int stages, int spc) {
   return s.tmem_slot + 16 + 1024;  // + alignment slack
 }
 
+// RN32(a / b) for a >= 0 and the constant divisors b = 6 (NVFP4) and 7 (INT4):
+// one multiply by c = RN32(1 / b), the exact remainder a - q0 b in one FMA, and
+// one correction q0 + rem c rounded once (Markstein's correction step for a
+// division by a known divisor). For these two divisors this equals the IEEE
+// quotient for every float32 a whose quotient is normal (checked exhaustively
+// binade by binade on the CPU); where the quotient underflows, both are far
+// below the smallest E4M3 / FP16 scale and give scale code 0.
+template <int kB>
+__device__ __forceinline__ float div_by_const_rn(float a) {
+  static_assert(kB == 6 || kB == 7, "verified divisors only");
+  const float c = __uint_as_float(kB == 6 ? 0x3e2aaaabu : 0x3e124925u);  // RN32(1 / b)
+  const float q0 = __fmul_rn(a, c);
+  const float rem = __fmaf_rn(-q0, static_cast<float>(kB), a);
+  return __fmaf_rn(rem, c, q0);
+}
+
+// max(a, b, c) of three float32 values in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest magnitude of 8 float pairs, as a tree of three-input maxima.
+__device__ __forceinline__ float absmax16(const float2* v) {
+  const float a = max3f(fabsf(v[0].x), fabsf(v[0].y), fabsf(v[1].x));
+  const float b = max3f(fabsf(v[1].y), fabsf(v[2].x), fabsf(v[2].y));
+  const float c = max3f(fabsf(v[3].x), fabsf(v[3].y), fabsf(v[4].x));
+  const float d = max3f(fabsf(v[4].y), fabsf(v[5].x), fabsf(v[5].y));
+  const float e = max3f(fabsf(v[6].x), fabsf(v[6].y), fabsf(v[7].x));
+  return fmaxf(max3f(a, b, c), max3f(d, e, fabsf(v[7].y)));
+}
+
 template <int kFmt>  // 0: NVFP4 (E2M1, UE4M3 per 16), 1: INT4 (FP16 per 64)
 __global__ void __launch_bounds__(kQaThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -257,11 +290,8 @@ __global__ void __launch_bounds__(kQaThreads, 1)
         uint32_t sc[2];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          float amax = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            amax = fmaxf(amax, fmaxf(fabsf(xv[8 * g + j].x), fabsf(xv[8 * g + j].y)));
-          sc[g] = e4m3_code(__fdiv_rn(amax, 6.0f));
+          const float amax = absmax16(xv + 8 * g);
+          sc[g] = e4m3_code(div_by_const_rn<6>(amax));
           const float2 vr = lds_f2(table_u32 + 8 * sc[g]);  // (decoded scale, its reciprocal)
           const float2 rcp2 = make_float2(vr.y, vr.y);
           float2 y0[4], y1[4];
@@ -283,11 +313,9 @@ __global__ void __launch_bounds__(kQaThreads, 1)
           *reinterpret_cast<uint32_t*>(p.scales + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) = word;
         }
       } else {
-        float amax = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(xv[j].x), fabsf(xv[j].y)));
+        float amax = fmaxf(absmax16(xv), absmax16(xv + 8));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-        const __half hs = __float2half_rn(__fdiv_rn(amax, 7.0f));
+        const __half hs = __float2half_rn(div_by_const_rn<7>(amax));
         const float sval = __half2float(hs);
 #pragma unroll
         for (int w = 0; w < 4; ++w) code[w] = 0u;
