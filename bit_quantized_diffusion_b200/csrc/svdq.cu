@@ -479,7 +479,7 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   const bool pair = (d->gemm_pair_mode < 0 ? pair_auto : d->gemm_pair_mode != 0) && M > kGmBM;
   const int ctas = pair ? 2 : 1;
   const int b_rows = kGmBN / ctas;
-  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1, tm_y;
   const uint64_t kb = static_cast<uint64_t>(K / 64);
   if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, kGmBKBytes,
                     kGmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -492,11 +492,15 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
                     256, 256, 8, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
+    // xl1 [M, r] float32 in chunks of 32 columns x 128 rows, 128-byte swizzle
     if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2, N, r,
-                      static_cast<uint64_t>(N) * 2, 64, kGmLrK, CU_TENSOR_MAP_SWIZZLE_128B))
+                      static_cast<uint64_t>(N) * 2, 64, kGmLrK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xl1, r, M,
+                      static_cast<uint64_t>(r) * 4, kGmLrK, kGmBM, CU_TENSOR_MAP_SWIZZLE_128B))
       return SVDQ_ERR_CUDA;
   } else {
     tm_l2 = tm_a;
+    tm_xl1 = tm_a;
   }
   // output: 32 x 32 boxes, bf16 rows of 64 B (64-byte swizzle) or f32 rows of 128 B
   const bool f32 = out == SVDQ_OUT_F32;
@@ -509,7 +513,6 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.N = N;
   p.K = K;
   p.r = r;
-  p.xl1 = xl1;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.out_f32 = f32;
   p.status = d->status;
@@ -520,9 +523,11 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
       pair ? launch_kernel(d, w4a4_nvfp4_gemm_kernel<true>, dim3(units * 2), dim3(kGmThreads),
-                           GmCfg<true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y, p)
+                           GmCfg<true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
+                           tm_y, p)
            : launch_kernel(d, w4a4_nvfp4_gemm_kernel<false>, dim3(units), dim3(kGmThreads),
-                           GmCfg<false>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_y, p);
+                           GmCfg<false>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
+                           tm_y, p);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;

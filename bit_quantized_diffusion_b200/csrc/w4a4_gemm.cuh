@@ -18,18 +18,34 @@
 //               across tiles through the ring
 //   warp 1      tensor-memory owner; in the leader CTA also the MMA issuer (one
 //               thread)
-//   warps 2-5   low-rank staging: xl1 (float32) as bf16 hi + lo operand tiles
+//   warps 2-5   one per tensor-memory lane quadrant: place each 4-bit slot's
+//               scale factors in tensor memory (tcgen05.st), and stage xl1
+//               (float32) as bf16 hi + lo operand tiles for the low-rank slots
 //   warps 6-13  epilogue, two warps per tensor-memory lane quadrant: accumulator
 //               -> + bias -> bf16 / f32 -> swizzled shared memory -> TMA store
 // Each tile is a sequence of ring slots: K/256 FP4 slots, then ceil(r/32)
-// low-rank slots holding an L2 chunk (by TMA) and the matching xl1 hi/lo tiles
-// (by the staging warps). A slot's "full" barrier (the leader's) counts the
+// low-rank slots holding an L2 chunk and the matching xl1 chunk [128 rows x 32]
+// float32 (both by TMA), which the quadrant warps turn in place into the bf16
+// hi + lo operand (each warp's 32 rows read and write the same 4 KB). A slot's "full" barrier (the leader's) counts the
 // leader's producer, whose expected bytes cover both CTAs' loads; a low-rank
 // slot's operand tiles are announced on the slot's "ready" barrier (the
 // leader's) by every staging warp of the pair; the MMA commit frees the slot
 // in both CTAs.
-// Two 256-column accumulators share tensor memory with a 64-column overlap
-// ([0, 256) and [192, 448)); scale factors sit in [448, 496). The epilogue
+// Scale factors: copying them into tensor memory with tcgen05.cp puts the copies
+// in the MMA issuer's queue, and they run serialised with the MMAs (three 512-byte
+// copies per 64-wide K block nearly double the time of its MMA). Instead the four
+// quadrant warps write them with tcgen05.st, which runs beside the MMAs: each warp
+// reads the slot's scale atoms from shared memory (each CTA loads its own copy,
+// announced on its own "sf landed" barrier) and stores the 32-lane pattern into
+// its own lane quadrant (every quadrant holds the same 32 lanes, the layout
+// tcgen05.cp .32x128b.warpx4 would produce). Two 48-column scale buffers
+// alternate between 4-bit slots: "sf full" (the leader's, counting every quadrant
+// warp of the pair) lets the MMA issuer in, "sf free" (committed after the slot's
+// MMAs) lets the warps refill the buffer. The MMA issuer is one thread whose
+// instruction latency paces the tensor pipe, so its loop is kept lean: operand
+// descriptors are built once and advanced by constant offsets.
+// Tensor-memory columns: two 256-column accumulators overlapping by 96 columns
+// ([0, 256) and [160, 416)), the two scale buffers in [416, 512). The epilogue
 // drains the overlapped columns of a tile first and releases them, so the next
 // tile's MMAs start while the rest of the tile is still being stored.
 #pragma once
@@ -48,8 +64,12 @@ constexpr int kGmSfaStage = 4 * 512;             // 4 atoms (one per 64-wide K b
 constexpr int kGmSfbStage = 2 * 4 * 512;         // 2 row blocks x 4 atoms
 constexpr int kGmLrK = 32;                       // low-rank K per ring slot
 constexpr int kGmLrATile = kGmBM * kGmLrK * 2;   // 8 KB per bf16 tile (hi, lo)
-// tensor-memory columns
-constexpr uint32_t kTmAcc1 = 192, kTmOverlap = 64, kTmSfa = 448, kTmSfb = 464, kTmCols = 512;
+// tensor-memory columns: accumulators at 0 and kTmAcc1 (kTmOverlap shared); scale
+// buffer b at kTmSf + kTmSfBuf b: 16 columns of A scales (4 per K block), then 32 of
+// B scales (8 per K block: two 128-row atoms of 4)
+constexpr uint32_t kTmAcc1 = 160, kTmOverlap = 96, kTmSf = 416, kTmSfBuf = 48, kTmCols = 512;
+static_assert(kTmAcc1 + 256 <= kTmSf && kTmSf + 2 * kTmSfBuf <= kTmCols, "tensor-memory layout");
+static_assert(256 - kTmOverlap == kTmAcc1, "the accumulators overlap by kTmOverlap columns");
 
 template <bool kPair>
 struct GmCfg {
@@ -62,7 +82,8 @@ struct GmCfg {
   static constexpr uint32_t kOut = kStages * kStageBytes;     // 1024-aligned
   static constexpr uint32_t kBias = kOut + kGmEpiWarps * kGmStageOut;
   static constexpr uint32_t kBars = kBias + kGmEpiWarps * 128 * 4;
-  static constexpr uint32_t kTmemSlot = kBars + 8 * (3 * kStages + 2);
+  // full, empty, ready, sf landed per stage; acc full, acc free; sf full, sf free per buffer
+  static constexpr uint32_t kTmemSlot = kBars + 8 * (4 * kStages + 2 + 2 * 2);
   static constexpr size_t kSmemBytes = kTmemSlot + 16 + 1024;
   static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert(kLrBTile + 2 * kGmLrATile <= kStageBytes, "a low-rank slot fits in a stage");
@@ -71,7 +92,6 @@ struct GmCfg {
 struct GemmParams {
   int M, N, K, r;
   int tiles_m, tiles;      // tiles of kCtas * 128 rows x 256 columns
-  const float* xl1;
   const __nv_bfloat16* bias;
   int out_f32;
   uint32_t* status;
@@ -84,6 +104,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                            const __grid_constant__ CUtensorMap tm_sfa,
                            const __grid_constant__ CUtensorMap tm_sfb,
                            const __grid_constant__ CUtensorMap tm_l2,
+                           const __grid_constant__ CUtensorMap tm_xl1,
                            const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   using Cfg = GmCfg<kPair>;
   constexpr int NS = Cfg::kStages;
@@ -117,8 +138,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   auto bar_full = [&](int s) { return sbase + Cfg::kBars + 8 * s; };
   auto bar_empty = [&](int s) { return sbase + Cfg::kBars + 8 * (NS + s); };
   auto bar_ready = [&](int s) { return sbase + Cfg::kBars + 8 * (2 * NS + s); };
-  const uint32_t bar_acc_full = sbase + Cfg::kBars + 8 * (3 * NS);
+  auto bar_sf_landed = [&](int s) { return sbase + Cfg::kBars + 8 * (3 * NS + s); };
+  const uint32_t bar_acc_full = sbase + Cfg::kBars + 8 * (4 * NS);
   const uint32_t bar_acc_free = bar_acc_full + 8;
+  auto bar_sf_full = [&](int b) { return bar_acc_full + 16 + 8 * b; };
+  auto bar_sf_free = [&](int b) { return bar_acc_full + 32 + 8 * b; };
   // the leader's copies of the pipeline barriers, as seen from this CTA
   auto lead = [&](uint32_t a) { return kPair ? map_peer_smem(a, 0) : a; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kTmemSlot);
@@ -128,16 +152,24 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       mbar_init(bar_full(s), 1);                  // leader producer (with tx)
       mbar_init(bar_ready(s), 4 * Cfg::kCtas);    // staging warps of a low-rank slot
       mbar_init(bar_empty(s), 1);
+      mbar_init(bar_sf_landed(s), 1);             // this CTA's producer (with tx)
     }
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_free, kGmEpiWarps * Cfg::kCtas);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_sf_full(b), 4 * Cfg::kCtas);  // quadrant warps of the pair
+      mbar_init(bar_sf_free(b), 1);               // MMA commit
+    }
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_sfa);
     prefetch_tmap(&tm_sfb);
     prefetch_tmap(&tm_y);
-    if (p.r > 0) prefetch_tmap(&tm_l2);
+    if (p.r > 0) {
+      prefetch_tmap(&tm_l2);
+      prefetch_tmap(&tm_xl1);
+    }
   }
   if (warp == 1) {
     if (kPair) {
@@ -177,18 +209,26 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           };
           if (kt < ktiles) {
             if (leader)
-              mbar_arrive_expect_tx(bar_full(s),
-                                    Cfg::kCtas * (kGmAStage + Cfg::kBStage + kGmSfaStage + kGmSfbStage));
+              mbar_arrive_expect_tx(bar_full(s), Cfg::kCtas * (kGmAStage + Cfg::kBStage));
             load(a_st(s), &tm_a, kt * kGmBKBytes, mrow);
             load(b_st(s), &tm_b, kt * kGmBKBytes, nrow);
-            // scale atoms viewed as rows of 256 B: 4 atoms = 8 rows
-            load(sfa_st(s), &tm_sfa, 0, ((mrow / 128) * kblocks + 4 * kt) * 2);
+            // scale atoms, viewed as rows of 256 B (4 atoms = 8 rows): this CTA's
+            // own copy, for its quadrant warps, on its own barrier
+            const uint32_t sl = bar_sf_landed(s);
+            mbar_arrive_expect_tx(sl, kGmSfaStage + kGmSfbStage);
+            tma_load_2d(sfa_st(s), &tm_sfa, sl, 0, ((mrow / 128) * kblocks + 4 * kt) * 2);
             for (int j = 0; j < 2; ++j)
-              load(sfb_st(s) + j * 2048, &tm_sfb, 0, ((n0 / 128 + j) * kblocks + 4 * kt) * 2);
+              tma_load_2d(sfb_st(s) + j * 2048, &tm_sfb, sl, 0, ((n0 / 128 + j) * kblocks + 4 * kt) * 2);
           } else {
-            // low-rank slot: L2 rows [32 c, 32 c + 32) x this CTA's columns, 64-wide
-            // boxes (rows past r read as zero)
+            // low-rank slot: xl1 rows of this CTA x columns [32 c, 32 c + 32), float32
+            // with 128-byte swizzle (rows past M and columns past r read as zero), on
+            // this CTA's own barrier for its quadrant warps
             const int c = kt - ktiles;
+            const uint32_t sl = bar_sf_landed(s);
+            mbar_arrive_expect_tx(sl, kGmBM * kGmLrK * 4);
+            tma_load_2d(stage(s) + Cfg::kLrBTile, &tm_xl1, sl, c * kGmLrK, mrow);
+            // L2 rows [32 c, 32 c + 32) x this CTA's columns, 64-wide boxes (rows
+            // past r read as zero)
             if (leader) mbar_arrive_expect_tx(bar_full(s), kGmLrK * kGmBN * 2);
             for (int nb = 0; nb < Cfg::kBRows / 64; ++nb)
               load(stage(s) + nb * (kGmLrK * 128), &tm_l2, nrow + nb * 64, c * kGmLrK);
@@ -204,6 +244,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const uint32_t id_lr = idesc_bf16_f32(mma_m, kGmBN, false, true);
       const uint32_t id_fp4 = idesc_nvfp4(mma_m, kGmBN);
       int kt_global = 0;
+      int fp4 = 0;           // 4-bit slots issued so far: fp4 & 1 is the scale buffer
+      // operand descriptors of ring stage 0; stage s is kStageBytes further (>> 4)
+      const uint64_t a_desc0 = smem_desc(a_st(0), 16, 1024, kSwizzle128B);
+      const uint64_t b_desc0 = smem_desc(b_st(0), 16, 1024, kSwizzle128B);
+      constexpr uint64_t kStageStep = static_cast<uint64_t>(Cfg::kStageBytes >> 4);
       uint32_t lr_uses = 0;  // bit s: parity of the low-rank uses of ring slot s so far
       for (int i = 0; i < my_tiles && ok; ++i) {
         const uint32_t acc = tmem + ((i & 1) ? kTmAcc1 : 0u);
@@ -219,32 +264,42 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           if (!ok) break;
           tc_fence_after();
           if (kt < ktiles) {
-            const int nkb = min(4, kblocks - 4 * kt);
-            for (int kb = 0; kb < nkb; ++kb) {
-              const uint64_t da = smem_desc(sfa_st(s) + kb * 512, 128, 128, kSwizzleNone);
-              const uint64_t db0 = smem_desc(sfb_st(s) + kb * 512, 128, 128, kSwizzleNone);
-              const uint64_t db1 = smem_desc(sfb_st(s) + 2048 + kb * 512, 128, 128, kSwizzleNone);
+            // this slot's scale factors are in tensor memory (both CTAs)
+            const uint32_t buf = static_cast<uint32_t>(fp4 & 1);
+            ok = mbar_wait(bar_sf_full(buf), (fp4 >> 1) & 1, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t sfa = tmem + kTmSf + kTmSfBuf * buf, sfb = sfa + 16;
+            const uint64_t ad = a_desc0 + kStageStep * static_cast<uint64_t>(s);
+            const uint64_t bd = b_desc0 + kStageStep * static_cast<uint64_t>(s);
+            const uint32_t acc0 = kt > 0 ? 1u : 0u;
+            // K block kb starts 32 bytes (2 in descriptor units) further along the row
+            if (kblocks - 4 * kt >= 4) {
               if (kPair) {
-                tc_cp_32x128b_warpx4_pair(tmem + kTmSfa + 4 * kb, da);
-                tc_cp_32x128b_warpx4_pair(tmem + kTmSfb + 8 * kb, db0);
-                tc_cp_32x128b_warpx4_pair(tmem + kTmSfb + 8 * kb + 4, db1);
+                mma_nvfp4_pair(acc, ad, bd, id_fp4, sfa, sfb, acc0);
+                mma_nvfp4_pair(acc, ad + 2, bd + 2, id_fp4, sfa + 4, sfb + 8, 1u);
+                mma_nvfp4_pair(acc, ad + 4, bd + 4, id_fp4, sfa + 8, sfb + 16, 1u);
+                mma_nvfp4_pair(acc, ad + 6, bd + 6, id_fp4, sfa + 12, sfb + 24, 1u);
               } else {
-                tc_cp_32x128b_warpx4(tmem + kTmSfa + 4 * kb, da);
-                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb, db0);
-                tc_cp_32x128b_warpx4(tmem + kTmSfb + 8 * kb + 4, db1);
+                mma_nvfp4(acc, ad, bd, id_fp4, sfa, sfb, acc0);
+                mma_nvfp4(acc, ad + 2, bd + 2, id_fp4, sfa + 4, sfb + 8, 1u);
+                mma_nvfp4(acc, ad + 4, bd + 4, id_fp4, sfa + 8, sfb + 16, 1u);
+                mma_nvfp4(acc, ad + 6, bd + 6, id_fp4, sfa + 12, sfb + 24, 1u);
+              }
+            } else {
+              const int nkb = kblocks - 4 * kt;
+              for (int kb = 0; kb < nkb; ++kb) {
+                const uint32_t accum = (kt > 0 || kb > 0) ? 1u : 0u;
+                if (kPair)
+                  mma_nvfp4_pair(acc, ad + 2 * kb, bd + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb, accum);
+                else
+                  mma_nvfp4(acc, ad + 2 * kb, bd + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb, accum);
               }
             }
-            for (int kb = 0; kb < nkb; ++kb) {
-              const uint64_t ad = smem_desc(a_st(s) + kb * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(b_st(s) + kb * 32, 16, 1024, kSwizzle128B);
-              const uint32_t accum = (kt > 0 || kb > 0) ? 1u : 0u;
-              if (kPair)
-                mma_nvfp4_pair(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
-                               accum);
-              else
-                mma_nvfp4(acc, ad, bd, id_fp4, tmem + kTmSfa + 4 * kb, tmem + kTmSfb + 8 * kb,
-                          accum);
-            }
+            // the scale buffer is free once this slot's MMAs are done
+            if (kPair) tc_commit_pair(bar_sf_free(buf), 0x3);
+            else tc_commit(bar_sf_free(buf));
+            ++fp4;
           } else {
             ok = mbar_wait(bar_ready(s), (lr_uses >> s) & 1u, p.status);
             lr_uses ^= 1u << s;
@@ -253,13 +308,14 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             // low-rank slot: B = L2 chunk (MN-major, 128-byte swizzle; 64-wide N
             // blocks 4096 B apart = LBO, 8-deep K groups 1024 B apart = SBO);
             // A = xl1 hi / lo (no-swizzle K-major: K-adjacent core matrices 128 B
-            // apart = LBO, 8-row groups 512 B apart = SBO)
-            const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
+            // apart = LBO; each 8-row group holds 512 B of hi, then 512 B of lo, so
+            // groups are 1024 B apart = SBO)
+            const uint32_t a_lr = stage(s) + Cfg::kLrBTile;
 #pragma unroll
             for (int kk = 0; kk < kGmLrK / 16; ++kk) {
               const uint64_t bd = smem_desc(stage(s) + kk * 2048, kGmLrK * 128, 1024, kSwizzle128B);
-              const uint64_t ah = smem_desc(a_hi + kk * 256, 128, 512, kSwizzleNone);
-              const uint64_t al = smem_desc(a_lo + kk * 256, 128, 512, kSwizzleNone);
+              const uint64_t ah = smem_desc(a_lr + kk * 256, 128, 1024, kSwizzleNone);
+              const uint64_t al = smem_desc(a_lr + 512 + kk * 256, 128, 1024, kSwizzleNone);
               if (kPair) {
                 mma_f16_pair(acc, ah, bd, id_lr, 1u);
                 mma_f16_pair(acc, al, bd, id_lr, 1u);
@@ -277,36 +333,72 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       }
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ low-rank staging
+    // ---------------------------------------- scale factors and low-rank staging
     const int quad = warp & 3;
     const int trow = quad * 32 + lane;
+    const uint32_t sf_lanes = tmem + kTmSf + (static_cast<uint32_t>(quad * 32) << 16);
     bool ok = true;
     int kt_global = 0;
+    int fp4 = 0;  // 4-bit slots handled so far: fp4 & 1 is the scale buffer
     for (int i = 0; i < my_tiles && ok; ++i) {
-      int m0, n0;
-      tile_mn(i, m0, n0);
-      const int m = m0 + kGmBM * static_cast<int>(rank) + trow;
-      // FP4 slots need nothing from the staging warps, but their "empty" phases
-      // are still waited in order: a parity wait is only meaningful one phase
-      // at a time, so skipping ahead could pass a phase that has not come yet.
-      for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global)
-        ok = mbar_wait(bar_empty(kt_global % NS), ((kt_global / NS) & 1) ^ 1, p.status);
+      // 4-bit slots: place the scale factors. The slot's "empty" phases are still
+      // waited in order: a parity wait is only meaningful one phase at a time, so
+      // skipping ahead could pass a phase that has not come yet.
+      for (int kt = 0; kt < ktiles && ok; ++kt, ++kt_global, ++fp4) {
+        const int s = kt_global % NS;
+        const int buf = fp4 & 1;
+        ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status) &&
+             mbar_wait(bar_sf_landed(s), (kt_global / NS) & 1, p.status);
+        // lane l: the 16 bytes at l * 16 of each scale atom (rows l, l + 32, l + 64,
+        // l + 96 of its 128-row block, 4 scales each) -> 4 columns per atom; read
+        // before waiting for the buffer
+        uint32_t sa[16], sbv[32];
+        if (ok) {
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 a = lds_u4(sfa_st(s) + kb * 512 + lane * 16);
+            sa[4 * kb] = a.x; sa[4 * kb + 1] = a.y; sa[4 * kb + 2] = a.z; sa[4 * kb + 3] = a.w;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint4 v = lds_u4(sfb_st(s) + j * 2048 + kb * 512 + lane * 16);
+              sbv[8 * kb + 4 * j] = v.x; sbv[8 * kb + 4 * j + 1] = v.y;
+              sbv[8 * kb + 4 * j + 2] = v.z; sbv[8 * kb + 4 * j + 3] = v.w;
+            }
+          }
+        }
+        ok = ok && (fp4 < 2 || mbar_wait(bar_sf_free(buf), ((fp4 >> 1) - 1) & 1, p.status));
+        ok = __all_sync(0xffffffffu, ok);  // tcgen05.st below needs the whole warp
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dst = sf_lanes + kTmSfBuf * static_cast<uint32_t>(buf);
+        tmem_st16(dst, sa);
+        tmem_st32(dst + 16, sbv);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          // the pair's MMAs read this CTA's scale columns through this SM's own
+          // tensor core: the completed stores are ordered for them by the fence
+          // and a CTA-scope release, as for the low-rank operand tiles
+          if (kPair) mbar_arrive_remote(lead(bar_sf_full(buf)));
+          else mbar_arrive(bar_sf_full(buf));
+        }
+      }
       for (int c = 0; c < lr_chunks && ok; ++c, ++kt_global) {
         const int s = kt_global % NS;
-        // load before waiting: the global read overlaps the wait for the slot
-        float v[kGmLrK];
-        const float4* src = reinterpret_cast<const float4*>(p.xl1 + static_cast<size_t>(m) * p.r +
-                                                            c * kGmLrK);
-#pragma unroll
-        for (int j = 0; j < kGmLrK / 4; ++j) {
-          // rows past M and columns past r (r % 32 == 16) contribute zeros
-          const float4 f = (m < p.M && c * kGmLrK + 4 * j < p.r) ? __ldg(src + j)
-                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
-        }
-        ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status);
+        ok = mbar_wait(bar_empty(s), ((kt_global / NS) & 1) ^ 1, p.status) &&
+             mbar_wait(bar_sf_landed(s), (kt_global / NS) & 1, p.status);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        const uint32_t a_hi = stage(s) + Cfg::kLrBTile, a_lo = a_hi + kGmLrATile;
+        // this lane's row of the float32 chunk (128 B, 16-byte units swizzled by row % 8)
+        const uint32_t lr = stage(s) + Cfg::kLrBTile;
+        float v[kGmLrK];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 f = lds_f4(lr + trow * 128 + ((q ^ (trow & 7)) << 4));
+          v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+        }
+        __syncwarp();  // the warp's 4 KB is read before any lane overwrites it
 #pragma unroll
         for (int cm = 0; cm < kGmLrK / 8; ++cm) {
           uint32_t hi[4], lo[4];
@@ -319,11 +411,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
             lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
           }
-          const uint32_t off = (trow >> 3) * 512 + cm * 128 + (trow & 7) * 16;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi + off), "r"(hi[0]),
+          const uint32_t off = (trow >> 3) * 1024 + cm * 128 + (trow & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lr + off), "r"(hi[0]),
                        "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
                        : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo + off), "r"(lo[0]),
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lr + off + 512), "r"(lo[0]),
                        "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
                        : "memory");
         }
@@ -357,12 +449,22 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       const int mrow = m0 + kGmBM * static_cast<int>(rank);
       const bool odd = i & 1;
       const uint32_t t_row = tmem + (odd ? kTmAcc1 : 0u) + (static_cast<uint32_t>(quad * 32) << 16);
-      // sub-tile order: the overlapped one, then three of the six others
+      // sub-tile order: the overlapped ones first (two in the first half's warps,
+      // one in the second's), then the five others
       int sub_col[4];
       const int ovl = odd ? 0 : kGmBN - kTmOverlap;   // first overlapped column
-      sub_col[0] = ovl + 32 * half;
       const int other0 = odd ? kTmOverlap : 0;        // first non-overlapped column
-      for (int t = 0; t < 3; ++t) sub_col[1 + t] = other0 + 32 * (3 * half + t);
+      if (half == 0) {
+        sub_col[0] = ovl;
+        sub_col[1] = ovl + 64;
+        sub_col[2] = other0;
+        sub_col[3] = other0 + 32;
+      } else {
+        sub_col[0] = ovl + 32;
+        sub_col[1] = other0 + 64;
+        sub_col[2] = other0 + 96;
+        sub_col[3] = other0 + 128;
+      }
       // bias for this warp's sub-tiles, fetched before the accumulator is ready
       __syncwarp();
 #pragma unroll
@@ -374,11 +476,18 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       ok = mbar_wait(bar_acc_full, i & 1, p.status);
       if (!ok) break;
       tc_fence_after();
+      uint32_t acc_next[32];  // the first half's second overlapped sub-tile
       for (int t = 0; t < 4; ++t) {
         const int j0 = sub_col[t];
         uint32_t acc[32];
-        tmem_ld32(t_row + j0, acc);
-        tmem_ld_wait();
+        if (t == 1 && half == 0) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) acc[q] = acc_next[q];
+        } else {
+          tmem_ld32(t_row + j0, acc);
+          if (t == 0 && half == 0) tmem_ld32(t_row + sub_col[1], acc_next);
+          tmem_ld_wait();
+        }
         if (t == 0) {
           // this warp's overlapped columns are in registers: let the next tile's MMAs in
           tc_fence_before();
