@@ -95,6 +95,59 @@ def quantize_int4(xhat: np.ndarray):
     return q.reshape(xhat.shape).astype(np.int8), np.where(zero, 0.0, s)
 
 
+# ------------------------------------------- two-level NVFP4 (per-tensor scale)
+# The NVFP4 format named on the pages (Diffusers blog, "quantization_config":
+# precision nvfp4, group_size 16) has a second scale level above the E4M3 group
+# scales: one float32 factor per tensor, so that a tensor whose range lies outside
+# what E4M3 group scales reach (amax/6 above 448 or below 2^-9) still quantizes
+# with the format's relative precision. The pages state no formula for it; the
+# reading (recorded in the design notes) is the usual one:
+#
+#   s_t  = RN32(amax / (6 * 448)) if that is a normal float32, else 1
+#   inv  = RN32(1 / s_t)
+#   x'   = RN32(x_hat * inv), then the one-level NVFP4 quantization of x'
+#   Y    = RN32(s_t,a * s_t,w) * (4-bit product) + (x_hat L1) L2 + bias
+#
+# with amax the largest |x_hat| of the tensor (x_hat = the smoothed activation;
+# the residual weight for weights). The low-rank branch keeps x_hat unscaled.
+
+NVFP4_TENSOR_RANGE = 6.0 * 448.0
+_F32_MIN_NORMAL = 2.0 ** -126
+
+
+def tensor_scale(xhat: np.ndarray):
+    """(s_t, inv) of a float32-valued tensor, both float32 values as float64."""
+    amax = float(np.max(np.abs(np.asarray(xhat, np.float64)))) if np.size(xhat) else 0.0
+    s = float(rn32(np.float64(amax) / NVFP4_TENSOR_RANGE))
+    if not s >= _F32_MIN_NORMAL:
+        s = 1.0
+    return s, float(rn32(np.float64(1.0) / s))
+
+
+def quantize_nvfp4_two_level(xhat: np.ndarray, inv: float):
+    """Two-level NVFP4: the one-level quantization of RN32(x_hat * inv)."""
+    return quantize_nvfp4(rn32(np.asarray(xhat, np.float64) * np.float64(inv)))
+
+
+def dequant_nvfp4_two_level(codes, s_code, s_t: float) -> np.ndarray:
+    return dequant_nvfp4(codes, s_code) * np.float64(s_t)
+
+
+def w4a4_linear_two_level(a_deq: np.ndarray, w_deq: np.ndarray, s_ta: float, s_tw: float,
+                          xl1: np.ndarray | None, L2: np.ndarray | None,
+                          bias: np.ndarray | None) -> np.ndarray:
+    """Y = RN32(s_ta * s_tw) * (a_deq @ w_deq^T) + xl1 @ L2 + bias, float64 (unrounded).
+
+    a_deq / w_deq are the one-level dequantized codes of the scaled tensors."""
+    alpha = float(rn32(np.float64(s_ta) * np.float64(s_tw)))
+    y = alpha * (np.asarray(a_deq, np.float64) @ np.asarray(w_deq, np.float64).T)
+    if xl1 is not None and L2 is not None and np.asarray(L2).shape[0] > 0:
+        y += np.asarray(xl1, np.float64) @ np.asarray(L2, np.float64)
+    if bias is not None:
+        y += np.asarray(bias, np.float64)[None, :]
+    return y
+
+
 def quantize(fmt: str, xhat: np.ndarray):
     if fmt == NVFP4:
         return quantize_nvfp4(xhat)
