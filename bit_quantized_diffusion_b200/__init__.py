@@ -177,6 +177,95 @@ def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int
     return Y
 
 
+def svdq_tensor_scale(X: torch.Tensor, smooth_inv: torch.Tensor | None = None,
+                      scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Two-level NVFP4: float32 [2] = (s_t, RN32(1 / s_t)) of x_hat = RN32(X * smooth_inv)."""
+    lib = N.load()
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bf16 tensor")
+    M, K = X.shape
+    if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
+        raise ValueError("smooth_inv must be float32 [K]")
+    if scale is None:
+        scale = torch.empty(2, dtype=torch.float32, device=X.device)
+    if scale.dtype != torch.float32 or scale.numel() < 2:
+        raise ValueError("scale must be float32 [2]")
+    N.check(lib.svdq_tensor_scale(M, K, _ptr(X), X.stride(0), _ptr(smooth_inv), _ptr(scale),
+                                  _stream(stream)), "svdq_tensor_scale")
+    return scale
+
+
+def svdq_quantize_act_two_level(X: torch.Tensor, scale: torch.Tensor, L1s: torch.Tensor | None = None,
+                                smooth_inv: torch.Tensor | None = None,
+                                codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                                xl1: torch.Tensor | None = None, stream=None):
+    """svdq_quantize_act in two-level NVFP4: codes and group scales of RN32(x_hat * scale[1]);
+    ``scale`` is the float32 [2] pair from svdq_tensor_scale. Returns (codes, scales, xl1)."""
+    lib = N.load()
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bf16 tensor")
+    if scale.dtype != torch.float32 or scale.numel() < 2:
+        raise ValueError("scale must be float32 [2]")
+    M, K = X.shape
+    r = 0 if L1s is None else L1s.shape[1]
+    f = N.NVFP4_G16
+    dev = X.device
+    if codes is None:
+        codes = torch.empty(lib.svdq_codes_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(lib.svdq_scales_bytes(f, M, K), dtype=torch.uint8, device=dev)
+    S = lib.svdq_xl1_splits(M, K, r) if r else 0
+    if r and xl1 is None:
+        xl1 = torch.empty((S, M, r), dtype=torch.float32, device=dev)
+    _need(codes, lib.svdq_codes_bytes(f, M, K), "codes")
+    _need(scales, lib.svdq_scales_bytes(f, M, K), "scales")
+    if L1s is not None and (L1s.dtype != torch.bfloat16 or tuple(L1s.shape) != (2, r, K)):
+        raise ValueError("L1s must be bf16 [2, r, K]")
+    if smooth_inv is not None and (smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K):
+        raise ValueError("smooth_inv must be float32 [K]")
+    if xl1 is not None and (xl1.dtype != torch.float32 or xl1.numel() < S * M * r):
+        raise ValueError(f"xl1 must be float32 [{S}, M, r]")
+    N.check(lib.svdq_quantize_act_two_level(M, K, r, _ptr(X), K, _ptr(smooth_inv), _ptr(scale),
+                                            _ptr(L1s), _ptr(codes), _ptr(scales),
+                                            _ptr(xl1) if r else None, _stream(stream)),
+            "svdq_quantize_act_two_level")
+    return codes, scales, (xl1.view(-1)[:M * r].view(M, r) if r else None)
+
+
+def svdq_w4a4_linear_two_level(a_codes, a_scales, a_tscale, xl1, w_codes, w_scales, w_tscale, L2,
+                               bias, M: int, N_: int, K: int, out_dtype=torch.bfloat16,
+                               Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Two-level NVFP4 W4A4 linear: Y = RN32(s_a s_w) * (4-bit product) + xl1 @ L2 + bias, with
+    a_tscale / w_tscale the float32 scale pairs of the activation and the weight."""
+    lib = N.load()
+    r = 0 if L2 is None else L2.shape[0]
+    if r and (xl1 is None or xl1.dtype != torch.float32 or xl1.numel() < M * r):
+        raise ValueError("xl1 must be float32 [M, r]")
+    for name, t in (("a_tscale", a_tscale), ("w_tscale", w_tscale)):
+        if t is None or t.dtype != torch.float32 or t.numel() < 1:
+            raise ValueError(f"{name} must be a float32 tensor scale pair")
+    out = N.OUT_F32 if out_dtype == torch.float32 else N.OUT_BF16
+    if Y is None:
+        Y = torch.empty((M, N_), dtype=out_dtype, device=a_codes.device)
+    if Y.dtype != out_dtype or Y.dim() != 2 or Y.shape[0] != M or Y.shape[1] < N_:
+        raise ValueError("Y must be [M, >= N] of out_dtype")
+    if L2 is not None and (L2.dtype != torch.bfloat16 or tuple(L2.shape) != (r, N_)):
+        raise ValueError("L2 must be bf16 [r, N]")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N_):
+        raise ValueError("bias must be bf16 [N]")
+    f = N.NVFP4_G16
+    _need(a_codes, lib.svdq_codes_bytes(f, M, K), "a_codes")
+    _need(a_scales, lib.svdq_scales_bytes(f, M, K), "a_scales")
+    _need(w_codes, lib.svdq_codes_bytes(f, N_, K), "w_codes")
+    _need(w_scales, lib.svdq_scales_bytes(f, N_, K), "w_scales")
+    N.check(lib.svdq_w4a4_linear_two_level(M, N_, K, r, _ptr(a_codes), _ptr(a_scales), _ptr(a_tscale),
+                                           _ptr(xl1) if r else None, _ptr(w_codes), _ptr(w_scales),
+                                           _ptr(w_tscale), _ptr(L2) if r else None, _ptr(bias),
+                                           _ptr(Y), Y.shape[1], out, _stream(stream)),
+            "svdq_w4a4_linear_two_level")
+    return Y
+
+
 def awq_w4a16_linear(X: torch.Tensor, qweight: torch.Tensor, sz: torch.Tensor,
                      bias: torch.Tensor | None, N_: int, group: int = 64,
                      Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -24,7 +24,8 @@ EXPORTS = (
     "awq_qweight_bytes", "awq_sz_bytes", "svdq_quantize_act", "svdq_w4a4_linear",
     "awq_w4a16_linear", "svdq_pack", "svdq_unpack", "svdq_check_device_status",
     "svdq_debug_wait_timeout", "svdq_pack_lowrank", "svdq_xl1_splits",
-    "svdq_quantize_act_noalloc",
+    "svdq_quantize_act_noalloc", "svdq_tensor_scale", "svdq_quantize_act_two_level",
+    "svdq_w4a4_linear_two_level",
 )
 
 _lib = None
@@ -60,6 +61,10 @@ def load() -> ctypes.CDLL:
         "svdq_pack_lowrank": (_I, [_I, _I, _P, _P, _P, _P]),
         "svdq_xl1_splits": (_I, [_I, _I, _I]),
         "svdq_quantize_act_noalloc": (_I, [_I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P]),
+        "svdq_tensor_scale": (_I, [_I, _I, _P, _I, _P, _P, _P]),
+        "svdq_quantize_act_two_level": (_I, [_I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
+        "svdq_w4a4_linear_two_level": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, _I, _I, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

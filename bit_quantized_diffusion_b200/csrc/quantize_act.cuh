@@ -58,6 +58,7 @@ struct QuantActParams {
   int spc;         // sub-chunks per stage (1 or 2)
   int m_pad;       // M rounded up to 128
   const float* smooth_inv;
+  const float* tensor_scale;  // NVFP4 two-level: [s_t, RN32(1 / s_t)] on the device, or null
   uint8_t* codes;
   uint8_t* scales;
   float* xl1;      // split 0 (and, after the reduction, the sum): [M][r]
@@ -238,6 +239,9 @@ __global__ void __launch_bounds__(kQaThreads, 1)
     const bool row_ok = m < p.M;
     uint8_t* const code_row = p.codes + static_cast<size_t>(m) * (p.K / 2) + half * 16;
     const uint32_t table_u32 = sbase + L.table;
+    // two-level NVFP4: the smoothed values are quantized as x_hat * RN32(1 / s_t)
+    const bool two_level = kFmt == 0 && p.tensor_scale != nullptr;
+    const float t_inv = two_level ? p.tensor_scale[1] : 1.0f;
     bool ok = true;
     int s = 0;        // ring slot of stage i
     uint32_t ph = 0;  // its phase parity
@@ -284,6 +288,11 @@ __global__ void __launch_bounds__(kQaThreads, 1)
       // this warp no longer reads the stage's shared memory
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty(slot));
+      if (two_level) {
+        const float2 t2 = make_float2(t_inv, t_inv);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xv[j] = __fmul2_rn(xv[j], t2);
+      }
       // -- a2 + a3: group scale and codes
       uint32_t code[4];
       if (kFmt == 0) {
@@ -391,6 +400,48 @@ __global__ void xl1_reduce_kernel(float4* xl1, const float4* rest, int splits, s
     }
     xl1[t] = v;
   }
+}
+
+// Largest |RN32(x * smooth_inv)| of an M x K bf16 tensor, accumulated into *amax_bits
+// (which holds float32 bits and starts at zero: non-negative floats order like
+// their bit patterns, so an integer atomic max is exact). Units of 8 columns.
+__global__ void tensor_absmax_kernel(const __nv_bfloat16* X, int ldx, const float* smooth_inv,
+                                     int M, int K, uint32_t* amax_bits) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int k8 = K / 8;
+  const size_t units = static_cast<size_t>(M) * k8;
+  float m = 0.0f;
+  for (size_t u = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(u / k8), c = static_cast<int>(u % k8) * 8;
+    const uint4 v = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * ldx + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+      if (smooth_inv != nullptr) {
+        a = __fmul_rn(a, smooth_inv[c + 2 * j]);
+        b = __fmul_rn(b, smooth_inv[c + 2 * j + 1]);
+      }
+      m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+    }
+  }
+  uint32_t bits = __float_as_uint(m);
+  bits = __reduce_max_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, bits);
+}
+
+// scale[0] = s_t = RN32(amax / (6 * 448)) if that is a normal float32, else 1;
+// scale[1] = RN32(1 / s_t). scale[0] holds the absolute maximum's bits on entry.
+__global__ void tensor_scale_finalize_kernel(float* scale) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const float amax = __uint_as_float(*reinterpret_cast<const uint32_t*>(scale));
+  float st = __fdiv_rn(amax, 2688.0f);
+  if (!(st >= 1.17549435e-38f)) st = 1.0f;  // 2^-126, the smallest normal float32
+  scale[0] = st;
+  scale[1] = __frcp_rn(st);
 }
 
 // L1s = diag(smooth_inv) L1 as two bf16 planes [2][r][K] (hi, lo): hi = RN_bf16(v),

@@ -300,8 +300,12 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
 
 svdq_status quantize_act_impl(svdq_format format, int M, int K, int r, const void* X, int ldx,
                               const float* smooth_inv, const void* L1s, void* codes, void* scales,
-                              float* xl1, bool static_rest, svdq_stream_t stream) {
+                              float* xl1, bool static_rest, svdq_stream_t stream,
+                              const float* tensor_scale = nullptr) {
   if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+  if (tensor_scale != nullptr && format != SVDQ_NVFP4_G16) return SVDQ_ERR_INVALID_ARG;
+  if (tensor_scale != nullptr && (reinterpret_cast<uintptr_t>(tensor_scale) & 7u))
+    return SVDQ_ERR_ALIGNMENT;
   if (M < 1 || K < 64 || K % 64 || !rank_ok(r) || ldx < K) return SVDQ_ERR_INVALID_ARG;
   if (X == nullptr || codes == nullptr || scales == nullptr) return SVDQ_ERR_INVALID_ARG;
   if ((r > 0) != (L1s != nullptr) || (r > 0) != (xl1 != nullptr)) return SVDQ_ERR_INVALID_ARG;
@@ -355,6 +359,7 @@ svdq_status quantize_act_impl(svdq_format format, int M, int K, int r, const voi
   p.spc = spc;
   p.m_pad = static_cast<int>(pad128(M));
   p.smooth_inv = smooth_inv;
+  p.tensor_scale = tensor_scale;
   p.codes = static_cast<uint8_t*>(codes);
   p.scales = static_cast<uint8_t*>(scales);
   // splits 1 .. S-1: the rest of the caller's buffer, or the library's static
@@ -450,11 +455,21 @@ svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, c
                            stream);
 }
 
-svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
+}  // extern "C"
+
+namespace {
+
+svdq_status w4a4_linear_impl(svdq_format format, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
                              const void* w_scales, const void* L2, const void* bias, void* Y,
-                             int ldy, svdq_out out, svdq_stream_t stream) {
+                             int ldy, svdq_out out, svdq_stream_t stream, const float* a_tscale,
+                             const float* w_tscale) {
   if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+  if ((a_tscale != nullptr) != (w_tscale != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (a_tscale != nullptr && format != SVDQ_NVFP4_G16) return SVDQ_ERR_INVALID_ARG;
+  if (a_tscale != nullptr && ((reinterpret_cast<uintptr_t>(a_tscale) & 3u) ||
+                              (reinterpret_cast<uintptr_t>(w_tscale) & 3u)))
+    return SVDQ_ERR_ALIGNMENT;
   if (out != SVDQ_OUT_BF16 && out != SVDQ_OUT_F32) return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || N < 16 || N % 16 || K < 64 || K % 64 || !rank_ok(r) || ldy < N)
     return SVDQ_ERR_INVALID_ARG;
@@ -514,6 +529,8 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
   p.K = K;
   p.r = r;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.a_tscale = a_tscale;
+  p.w_tscale = w_tscale;
   p.out_f32 = f32;
   p.status = d->status;
   p.tiles_m = (M + kGmBM * ctas - 1) / (kGmBM * ctas);
@@ -533,6 +550,64 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
     return SVDQ_ERR_CUDA;
   }
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, const void* a_codes,
+                             const void* a_scales, const float* xl1, const void* w_codes,
+                             const void* w_scales, const void* L2, const void* bias, void* Y,
+                             int ldy, svdq_out out, svdq_stream_t stream) {
+  return w4a4_linear_impl(format, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales, L2, bias,
+                          Y, ldy, out, stream, nullptr, nullptr);
+}
+
+svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a_codes,
+                                       const void* a_scales, const float* a_tensor_scale,
+                                       const float* xl1, const void* w_codes, const void* w_scales,
+                                       const float* w_tensor_scale, const void* L2, const void* bias,
+                                       void* Y, int ldy, svdq_out out, svdq_stream_t stream) {
+  if (a_tensor_scale == nullptr || w_tensor_scale == nullptr) return SVDQ_ERR_INVALID_ARG;
+  return w4a4_linear_impl(SVDQ_NVFP4_G16, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales,
+                          L2, bias, Y, ldy, out, stream, a_tensor_scale, w_tensor_scale);
+}
+
+svdq_status svdq_tensor_scale(int M, int K, const void* X, int ldx, const float* smooth_inv,
+                              float* scale, svdq_stream_t stream) {
+  if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8 || !X || !scale) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(scale) & 7u) ||
+      (smooth_inv && !aligned16(smooth_inv)))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scale, 0, sizeof(float), cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  const size_t units = static_cast<size_t>(M) * (K / 8);
+  unsigned grid = grid_for(units, 256);
+  if (grid > static_cast<unsigned>(4 * d->num_sms)) grid = 4 * d->num_sms;
+  if (launch_kernel(d, tensor_absmax_kernel, dim3(grid), dim3(256), 0, cs, 1,
+                    static_cast<const __nv_bfloat16*>(X), ldx, smooth_inv, M, K,
+                    reinterpret_cast<uint32_t*>(scale)) != cudaSuccess ||
+      launch_kernel(d, tensor_scale_finalize_kernel, dim3(1), dim3(1), 0, cs, 1, scale) !=
+          cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+svdq_status svdq_quantize_act_two_level(int M, int K, int r, const void* X, int ldx,
+                                        const float* smooth_inv, const float* tensor_scale,
+                                        const void* L1s, void* codes, void* scales, float* xl1,
+                                        svdq_stream_t stream) {
+  if (tensor_scale == nullptr) return SVDQ_ERR_INVALID_ARG;
+  return quantize_act_impl(SVDQ_NVFP4_G16, M, K, r, X, ldx, smooth_inv, L1s, codes, scales, xl1,
+                           false, stream, tensor_scale);
 }
 
 svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, const void* qweight,

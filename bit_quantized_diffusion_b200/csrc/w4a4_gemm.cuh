@@ -93,6 +93,10 @@ struct GemmParams {
   int M, N, K, r;
   int tiles_m, tiles;      // tiles of kCtas * 128 rows x 256 columns
   const __nv_bfloat16* bias;
+  // two-level NVFP4: the activation and weight tensor scales s_t (device), or null;
+  // Y = RN32(s_a s_w) * (4-bit product) + xl1 L2 + bias
+  const float* a_tscale;
+  const float* w_tscale;
   int out_f32;
   uint32_t* status;
 };
@@ -337,6 +341,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int quad = warp & 3;
     const int trow = quad * 32 + lane;
     const uint32_t sf_lanes = tmem + kTmSf + (static_cast<uint32_t>(quad * 32) << 16);
+    // two-level NVFP4: the low-rank branch shares the accumulator that the epilogue
+    // multiplies by alpha, so xl1 enters divided by it
+    const float alpha_inv =
+        p.a_tscale != nullptr ? __frcp_rn(__fmul_rn(p.a_tscale[0], p.w_tscale[0])) : 1.0f;
     bool ok = true;
     int kt_global = 0;
     int fp4 = 0;  // 4-bit slots handled so far: fp4 & 1 is the scale buffer
@@ -400,6 +408,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
         __syncwarp();  // the warp's 4 KB is read before any lane overwrites it
 #pragma unroll
+        for (int q = 0; q < kGmLrK; ++q) v[q] = __fmul_rn(v[q], alpha_inv);  // exact when 1
+#pragma unroll
         for (int cm = 0; cm < kGmLrK / 8; ++cm) {
           uint32_t hi[4], lo[4];
 #pragma unroll
@@ -443,6 +453,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const uint32_t free_bar = lead(bar_acc_free);
     bool ok = true;
     int stores = 0;
+    const float alpha = p.a_tscale != nullptr ? __fmul_rn(p.a_tscale[0], p.w_tscale[0]) : 1.0f;
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
@@ -502,11 +513,14 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         const float4* bv = reinterpret_cast<const float4*>(bias_s + t * 32);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
+          // y = alpha * acc + bias, one rounding (alpha = 1 without tensor scales: the
+          // plain sum); with two-level scales the accumulator holds the 4-bit product
+          // and the low-rank term divided by alpha
           const float4 b = bv[q4];
-          y[4 * q4 + 0] = __uint_as_float(acc[4 * q4 + 0]) + b.x;
-          y[4 * q4 + 1] = __uint_as_float(acc[4 * q4 + 1]) + b.y;
-          y[4 * q4 + 2] = __uint_as_float(acc[4 * q4 + 2]) + b.z;
-          y[4 * q4 + 3] = __uint_as_float(acc[4 * q4 + 3]) + b.w;
+          y[4 * q4 + 0] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 0]), alpha, b.x);
+          y[4 * q4 + 1] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 1]), alpha, b.y);
+          y[4 * q4 + 2] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 2]), alpha, b.z);
+          y[4 * q4 + 3] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 3]), alpha, b.w);
         }
         // stage the warp's 32 x 32 sub-tile in the TMA store's swizzled layout
         uint32_t buf;

@@ -180,6 +180,53 @@ svdq_status svdq_w4a4_linear(svdq_format format, int M, int N, int K, int r, con
                              int ldy, svdq_out out, svdq_stream_t stream);
 
 /*
+ * Two-level NVFP4. NVFP4 as named on the pages (Diffusers blog,
+ * "quantization_config": precision nvfp4, group_size 16: E2M1 values with one
+ * E4M3 scale per 16) has a second scale level above the group scales: one
+ * float32 factor s_t per tensor, which lets a tensor whose range E4M3 group
+ * scales cannot cover (amax / 6 above 448 or below 2^-9) keep the format's
+ * relative precision. The pages state no formula for it; this library uses
+ *
+ *   s_t = RN32(amax / (6 * 448)) if that is a normal float32, else 1
+ *   codes and group scales of x' = RN32(x_hat * RN32(1 / s_t)), exactly as
+ *   svdq_quantize_act does for x_hat
+ *   Y = RN32(s_t,a * s_t,w) * sum_g s_a s_w sum_k q_a q_w + xl1 L2 + bias
+ *
+ * svdq_tensor_scale -- scale[0] = s_t and scale[1] = RN32(1 / s_t) of
+ *   x_hat = RN32(X * smooth_inv) (smooth_inv NULL: x_hat = X).
+ *   X device bf16 [M, ldx], ldx % 8 == 0; smooth_inv device float32 [K] or NULL;
+ *   scale device float32 [2], 8-byte aligned, written. Enqueues a 4-byte memset
+ *   of scale[0] and two kernels (an absolute-maximum pass over X, then one thread).
+ *
+ * svdq_quantize_act_two_level -- svdq_quantize_act in NVFP4 with the codes and
+ *   group scales of x' = RN32(x_hat * scale[1]); xl1 = x_hat L1 is unchanged
+ *   (unscaled). scale: device float32 [2] as svdq_tensor_scale writes it (for the
+ *   same tensor, or a calibrated [s_t, RN32(1 / s_t)]), 8-byte aligned. Residual
+ *   weights are quantized the same way with smooth_inv NULL, r 0 and their own
+ *   scale. Other arguments as for svdq_quantize_act.
+ *
+ * svdq_w4a4_linear_two_level -- svdq_w4a4_linear in NVFP4 for codes from
+ *   svdq_quantize_act_two_level: a_tensor_scale and w_tensor_scale are the device
+ *   scale pairs of the activation and the weight (element 0, s_t, is read); alpha =
+ *   RN32(a_tensor_scale[0] * w_tensor_scale[0]). The low-rank term shares the
+ *   tensor-memory accumulator with the 4-bit product, so it enters as
+ *   RN32(xl1 * RN32(1 / alpha)) and the epilogue computes alpha * acc + bias (one
+ *   extra rounding of the low-rank term, relative 2^-24). Other arguments as for
+ *   svdq_w4a4_linear.
+ */
+svdq_status svdq_tensor_scale(int M, int K, const void* X, int ldx, const float* smooth_inv,
+                              float* scale, svdq_stream_t stream);
+svdq_status svdq_quantize_act_two_level(int M, int K, int r, const void* X, int ldx,
+                                        const float* smooth_inv, const float* scale,
+                                        const void* L1s, void* codes, void* scales, float* xl1,
+                                        svdq_stream_t stream);
+svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a_codes,
+                                       const void* a_scales, const float* a_tensor_scale,
+                                       const float* xl1, const void* w_codes, const void* w_scales,
+                                       const float* w_tensor_scale, const void* L2, const void* bias,
+                                       void* Y, int ldy, svdq_out out, svdq_stream_t stream);
+
+/*
  * awq_w4a16_linear -- step a7, the AWQ W4A16 linear for small-M modulation
  * projections (Diffusers blog, "From SVDQuant to Nunchaku Lite": awq_w4a16 for
  * the memory-bound adaptive-norm projections).
