@@ -438,6 +438,34 @@ def main() -> None:
     k3_ms = sum(b[1].elapsed_time(e) for b, e in zip(ev_k, ev_ke)) / args.steps
     status = bq.svdq_check_device_status()
 
+    # ------------------------------ two-level NVFP4 on the same layer (per-tensor scales)
+    # The same X and weights, quantized with a per-tensor float32 scale above the
+    # group scales: the tensor scale of the smoothed activation, the two-level
+    # quantizer and the two-level GEMM, each timed event to event after the flush.
+    w_tscale = bq.svdq_tensor_scale(svdq_w["R"])
+    wc2, ws2, _ = bq.svdq_quantize_act_two_level(svdq_w["R"], w_tscale)
+    a_tscale = torch.empty(2, dtype=torch.float32, device=dev)
+    codes2, scales2 = torch.empty_like(codes), torch.empty_like(scales)
+    xl1_2 = torch.empty_like(xl1)
+    Y2 = torch.empty_like(Y)
+    n2 = max(3, min(args.steps, 200))
+    ev2 = [[mk() for _ in range(4)] for _ in range(n2 + 3)]
+    for i in range(n2 + 3):
+        flush()
+        ev2[i][0].record(stream)
+        bq.svdq_tensor_scale(X, svdq_w["smooth_inv"], a_tscale, stream=stream)
+        ev2[i][1].record(stream)
+        _, _, xl1_view = bq.svdq_quantize_act_two_level(X, a_tscale, svdq_w["L1s"], svdq_w["smooth_inv"],
+                                                        codes=codes2, scales=scales2, xl1=xl1_2,
+                                                        stream=stream)
+        ev2[i][2].record(stream)
+        bq.svdq_w4a4_linear_two_level(codes2, scales2, a_tscale, xl1_view, wc2, ws2, w_tscale,
+                                      svdq_w["L2"], bias, M, N, K, Y=Y2, stream=stream)
+        ev2[i][3].record(stream)
+    torch.cuda.synchronize()
+    tl = [sum(e[j].elapsed_time(e[j + 1]) for e in ev2[3:]) / n2 for j in range(3)]
+    status = status or bq.svdq_check_device_status()
+
     # ----------------------------------------------- end to end, host buffers
     Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
     Xh.copy_(X)
@@ -543,6 +571,13 @@ def main() -> None:
             "awq_w4a16_linear_gbs": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / (k3_ms * 1e-3) / 1e9,
             "hbm_peak_gbs": peaks["hbm_gbs"],
             "cublas_bf16_tflops_same_shape": cublas_tflops,
+            "two_level_nvfp4": {
+                "timing": f"the same layer with per-tensor float32 scales, {n2} steps, event to event",
+                "svdq_tensor_scale_us": tl[0] * 1e3,
+                "svdq_quantize_act_two_level_us": tl[1] * 1e3,
+                "svdq_w4a4_linear_two_level_us": tl[2] * 1e3,
+                "svdq_w4a4_linear_two_level_tflops_4bit": k2_flops / (tl[2] * 1e-3) / 1e12,
+            },
         },
         "device_status": status,
     }

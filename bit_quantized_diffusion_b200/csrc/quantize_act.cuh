@@ -412,18 +412,23 @@ __global__ void tensor_absmax_kernel(const __nv_bfloat16* X, int ldx, const floa
   const int k8 = K / 8;
   const size_t units = static_cast<size_t>(M) * k8;
   float m = 0.0f;
+#pragma unroll 4
   for (size_t u = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; u < units;
        u += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int row = static_cast<int>(u / k8), c = static_cast<int>(u % k8) * 8;
-    const uint4 v = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * ldx + c);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * ldx + c));
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float sm[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+    if (smooth_inv != nullptr) {
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(smooth_inv + c));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(smooth_inv + c + 4));
+      sm[0] = s0.x; sm[1] = s0.y; sm[2] = s0.z; sm[3] = s0.w;
+      sm[4] = s1.x; sm[5] = s1.y; sm[6] = s1.z; sm[7] = s1.w;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
-      if (smooth_inv != nullptr) {
-        a = __fmul_rn(a, smooth_inv[c + 2 * j]);
-        b = __fmul_rn(b, smooth_inv[c + 2 * j + 1]);
-      }
+      const float a = __fmul_rn(__uint_as_float(w[j] << 16), sm[2 * j]);  // exact when 1
+      const float b = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), sm[2 * j + 1]);
       m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
     }
   }
