@@ -7,16 +7,26 @@ from __future__ import annotations
 
 import torch
 
-from . import (awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_scales_bytes,
-               svdq_w4a4_linear, svdq_xl1_splits)
+from . import (awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_quantize_act_two_level,
+               svdq_scales_bytes, svdq_tensor_scale, svdq_w4a4_linear, svdq_w4a4_linear_two_level,
+               svdq_xl1_splits)
 
 
 class SvdqW4A4Linear:
-    """Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + bias on prepared weights."""
+    """Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + bias on prepared weights.
 
-    def __init__(self, weights: dict, bias: torch.Tensor | None, max_tokens: int):
+    Weights prepared with a per-tensor scale (``w_tscale``) make the layer two-level
+    NVFP4: the activation's scale pair is ``act_scale`` (float32 [2], calibrated) or,
+    when that is None, computed on the device for every call."""
+
+    def __init__(self, weights: dict, bias: torch.Tensor | None, max_tokens: int,
+                 act_scale: torch.Tensor | None = None):
         self.w = weights
         self.bias = bias
+        self.two_level = weights.get("w_tscale") is not None
+        self.act_scale = act_scale
+        self._a_scale = (torch.empty(2, dtype=torch.float32, device=weights["w_codes"].device)
+                         if self.two_level else None)
         self.fmt = weights["fmt"]
         self.N, self.K, self.r = weights["N"], weights["K"], weights["r"]
         dev = weights["w_codes"].device
@@ -34,6 +44,16 @@ class SvdqW4A4Linear:
         if M > self.max_tokens:
             raise ValueError(f"{M} tokens > workspace for {self.max_tokens}")
         xl1 = self.xl1[:svdq_xl1_splits(M, self.K, self.r) * M * self.r] if self.r else None
+        if self.two_level:
+            a_scale = self.act_scale
+            if a_scale is None:
+                a_scale = svdq_tensor_scale(x, self.w["smooth_inv"], self._a_scale, stream=stream)
+            codes, scales, xl1 = svdq_quantize_act_two_level(
+                x, a_scale, self.w["L1s"], self.w["smooth_inv"], codes=self.codes, scales=self.scales,
+                xl1=xl1, stream=stream)
+            return svdq_w4a4_linear_two_level(codes, scales, a_scale, xl1, self.w["w_codes"],
+                                              self.w["w_scales"], self.w["w_tscale"], self.w["L2"],
+                                              self.bias, M, self.N, self.K, Y=y, stream=stream)
         codes, scales, xl1 = svdq_quantize_act(x, self.w["L1s"], self.w["smooth_inv"], fmt=self.fmt,
                                                codes=self.codes, scales=self.scales, xl1=xl1,
                                                stream=stream)

@@ -18,7 +18,8 @@ from __future__ import annotations
 
 import torch
 
-from . import svdq_pack, svdq_pack_lowrank, svdq_quantize_act
+from . import (svdq_pack, svdq_pack_lowrank, svdq_quantize_act, svdq_quantize_act_two_level,
+               svdq_tensor_scale)
 
 
 def smoothing(x_absmax: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
@@ -32,13 +33,17 @@ def smoothing(x_absmax: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
 
 
 def prepare_svdq_weights(w: torch.Tensor, x_absmax: torch.Tensor, rank: int,
-                         fmt: str = "nvfp4") -> dict:
+                         fmt: str = "nvfp4", two_level: bool = False) -> dict:
     """w [N, K] bf16 (nn.Linear layout), x_absmax [K] per-channel max |X|.
 
     Returns device tensors: smooth_inv [K] f32, L1 [K, r] bf16, L1s [2, r, K] bf16
     (the down-projection operand), L2 [r, N] bf16, w_codes, w_scales (tiled), and
-    R [N, K] bf16 (the quantized residual's input).
+    R [N, K] bf16 (the quantized residual's input). With ``two_level`` (NVFP4 only)
+    the residual is quantized with its own per-tensor scale, returned as w_tscale
+    (float32 [2]: s_t, 1 / s_t); otherwise w_tscale is None.
     """
+    if two_level and fmt != "nvfp4":
+        raise ValueError("two-level scaling is an NVFP4 format")
     N, K = w.shape
     smooth_inv = smoothing(x_absmax, w)
     w_hat = w.double() / smooth_inv.double()[None, :]
@@ -53,9 +58,16 @@ def prepare_svdq_weights(w: torch.Tensor, x_absmax: torch.Tensor, rank: int,
     else:
         L1 = L1s = L2 = None
         R = w_hat.to(torch.bfloat16)
-    w_codes, w_scales, _ = svdq_quantize_act(R.contiguous(), None, None, fmt=fmt)
+    R = R.contiguous()
+    if two_level:
+        w_tscale = svdq_tensor_scale(R)
+        w_codes, w_scales, _ = svdq_quantize_act_two_level(R, w_tscale)
+    else:
+        w_tscale = None
+        w_codes, w_scales, _ = svdq_quantize_act(R, None, None, fmt=fmt)
     return {"smooth_inv": smooth_inv.contiguous(), "L1": L1, "L1s": L1s, "L2": L2.contiguous() if L2 is not None else None,
-            "w_codes": w_codes, "w_scales": w_scales, "R": R, "fmt": fmt, "N": N, "K": K, "r": rank}
+            "w_codes": w_codes, "w_scales": w_scales, "w_tscale": w_tscale, "R": R, "fmt": fmt, "N": N,
+            "K": K, "r": rank}
 
 
 def prepare_awq_weights(w: torch.Tensor) -> dict:

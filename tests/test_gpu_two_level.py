@@ -123,3 +123,60 @@ def test_out_of_range_layer_matches_the_oracle(bq, M, N, K, r, out_f32):
     one = S.w4a4_linear(S.dequant_nvfp4(q1, s1), S.dequant_nvfp4(qw1, sw1), S.down_proj(x, L1), L2,
                         F.bf16_from_bits(bias_b))
     assert C.rel_l2(one, ref) > 0.05
+
+
+def test_layer_class_two_level_matches_the_oracle(bq):
+    """SvdqW4A4Linear in two-level mode (per-call activation scale) on weights
+    quantized two-level by the library, against the oracle's two-level layer."""
+    from bit_quantized_diffusion_b200.layers import SvdqW4A4Linear
+    shape = WL.custom_svdq("two_level_layer", 384, 1024, 512, 32, seed=33, n_outliers=8,
+                           outlier_scale=50.0, spike_rank=8, spike_sv=5.0)
+    layer = C.oracle_layer(shape)
+    si = C.f32_tensor(layer["smooth_inv"])
+    Rt = C.bf16_tensor(F.bf16_bits(layer["R"]))
+    w_tscale = bq.svdq_tensor_scale(Rt)
+    wc, ws, _ = bq.svdq_quantize_act_two_level(Rt, w_tscale)
+    weights = {"smooth_inv": si, "L1s": bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si),
+               "L2": C.bf16_tensor(F.bf16_bits(layer["L2"])), "w_codes": wc, "w_scales": ws,
+               "w_tscale": w_tscale, "fmt": "nvfp4", "N": shape.N, "K": shape.K, "r": shape.r}
+    lin = SvdqW4A4Linear(weights, C.bf16_tensor(layer["bias_bits"]), max_tokens=512)
+    y = lin(C.bf16_tensor(layer["x_bits"]))
+    assert bq.svdq_check_device_status() == 0
+    xhat = S.smooth(F.bf16_from_bits(layer["x_bits"]), layer["smooth_inv"])
+    sa, inva = S.tensor_scale(xhat)
+    sw, invw = S.tensor_scale(layer["R"])
+    qa, sca = S.quantize_nvfp4_two_level(xhat, inva)
+    qw, scw = S.quantize_nvfp4_two_level(layer["R"], invw)
+    ref = S.w4a4_linear_two_level(S.dequant_nvfp4(qa, sca), S.dequant_nvfp4(qw, scw), sa, sw,
+                                  S.down_proj(xhat, layer["L1"]), layer["L2"],
+                                  F.bf16_from_bits(layer["bias_bits"]))
+    C.assert_gemm_close(y.float().cpu().numpy().astype(np.float64), ref, bf16_out=True,
+                        what="two-level layer Y")
+
+
+def test_prep_two_level_weights(bq):
+    """prepare_svdq_weights(two_level=True): the residual's scale pair, codes and group
+    scales bit-exact against the oracle on the residual prep returns, and the layer it
+    makes (per-call activation scale) close to the unquantized product on weights too
+    small for E4M3 group scales alone."""
+    from bit_quantized_diffusion_b200 import prep
+    from bit_quantized_diffusion_b200.layers import SvdqW4A4Linear
+    rng = np.random.default_rng(51)
+    M, N, K, r = 256, 384, 512, 32
+    x = C.bf16_tensor(bf16_bits(rng.standard_normal((M, K)) * 3.0))
+    w = C.bf16_tensor(bf16_bits(rng.standard_normal((N, K)) * 1e-7))
+    wt = prep.prepare_svdq_weights(w, x.float().abs().amax(dim=0), r, "nvfp4", two_level=True)
+    R = C.bf16_bits_of(wt["R"])
+    Rd = F.bf16_from_bits(R)
+    s_w, inv_w = S.tensor_scale(Rd)
+    got = wt["w_tscale"].cpu().numpy().astype(np.float64)
+    assert (got[0], got[1]) == (s_w, inv_w)
+    q, sc = S.quantize_nvfp4_two_level(Rd, inv_w)
+    assert np.array_equal(wt["w_codes"].cpu().numpy(), S.pack_nibbles(q).reshape(-1))
+    assert np.array_equal(wt["w_scales"].cpu().numpy(), LO.tile_nvfp4_scales(sc))
+    y = SvdqW4A4Linear(wt, None, max_tokens=M)(x)
+    assert bq.svdq_check_device_status() == 0
+    want = x.double() @ w.double().T
+    assert float((y.double() - want).norm() / want.norm()) < 0.15
+    with pytest.raises(ValueError):
+        prep.prepare_svdq_weights(w, x.float().abs().amax(dim=0), r, "int4", two_level=True)
