@@ -466,6 +466,27 @@ def main() -> None:
     tl = [sum(e[j].elapsed_time(e[j + 1]) for e in ev2[3:]) / n2 for j in range(3)]
     status = status or bq.svdq_check_device_status()
 
+    # ------------------- the same layer as a fused QKV projection (norm + rotation epilogue)
+    # The QKV layer's 9216 columns are 24 heads each of Q, K and V; the GEMM with the
+    # per-head RMS norm of Q and K and the rotation by row-position angles in its
+    # epilogue, timed event to event after the flush, against the plain GEMM above.
+    qe = WL.qkv_epilogue_inputs(M, seed=SHAPE.seed + 100, angles="positions")
+    norm_q, norm_k = to_dev(qe["norm_q"]), to_dev(qe["norm_k"])
+    rope_cos = torch.from_numpy(qe["cos"]).to(dev)
+    rope_sin = torch.from_numpy(qe["sin"]).to(dev)
+    Y3 = torch.empty_like(Y)
+    ev3 = [[mk() for _ in range(2)] for _ in range(n2 + 3)]
+    for i in range(n2 + 3):
+        flush()
+        ev3[i][0].record(stream)
+        bq.svdq_w4a4_linear_qkv_norm_rope(codes, scales, xl1, svdq_w["w_codes"], svdq_w["w_scales"],
+                                          svdq_w["L2"], bias, norm_q, norm_k, rope_cos, rope_sin, M, N, K,
+                                          Y=Y3, stream=stream)
+        ev3[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_qkv = sum(e[0].elapsed_time(e[1]) for e in ev3[3:]) / n2
+    status = status or bq.svdq_check_device_status()
+
     # ----------------------------------------------- end to end, host buffers
     Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
     Xh.copy_(X)
@@ -577,6 +598,12 @@ def main() -> None:
                 "svdq_quantize_act_two_level_us": tl[1] * 1e3,
                 "svdq_w4a4_linear_two_level_us": tl[2] * 1e3,
                 "svdq_w4a4_linear_two_level_tflops_4bit": k2_flops / (tl[2] * 1e-3) / 1e12,
+            },
+            "fused_qkv_norm_rope": {
+                "timing": f"the same layer as Q, K, V of 24 heads of 128, per-head RMS norm of Q and K "
+                          f"and the pairwise rotation in the GEMM epilogue, {n2} steps, event to event",
+                "svdq_w4a4_linear_qkv_norm_rope_us": t_qkv * 1e3,
+                "svdq_w4a4_linear_qkv_norm_rope_tflops_4bit": k2_flops / (t_qkv * 1e-3) / 1e12,
             },
         },
         "device_status": status,

@@ -177,6 +177,47 @@ def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int
     return Y
 
 
+def svdq_w4a4_linear_qkv_norm_rope(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, norm_q,
+                                   norm_k, rope_cos, rope_sin, M: int, N_: int, K: int,
+                                   eps: float = 1e-6, out_dtype=torch.bfloat16,
+                                   Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The fused QKV projection (NVFP4): Y [M, N] = Q(X_hat) Q(R)^T + xl1 @ L2 + bias with
+    every 128-column head of Q and K (columns [0, N/3) and [N/3, 2N/3)) RMS-normalised
+    (norm_q / norm_k bf16 [128] or None, eps) and then turned pairwise by rope_cos /
+    rope_sin float32 [M, 64] (both None: no rotation); V unchanged. N % 384 == 0."""
+    lib = N.load()
+    r = 0 if L2 is None else L2.shape[0]
+    if r and (xl1 is None or xl1.dtype != torch.float32 or xl1.numel() < M * r):
+        raise ValueError("xl1 must be float32 [M, r]")
+    out = N.OUT_F32 if out_dtype == torch.float32 else N.OUT_BF16
+    if Y is None:
+        Y = torch.empty((M, N_), dtype=out_dtype, device=a_codes.device)
+    if Y.dtype != out_dtype or Y.dim() != 2 or Y.shape[0] != M or Y.shape[1] < N_:
+        raise ValueError("Y must be [M, >= N] of out_dtype")
+    if L2 is not None and (L2.dtype != torch.bfloat16 or tuple(L2.shape) != (r, N_)):
+        raise ValueError("L2 must be bf16 [r, N]")
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.numel() != N_):
+        raise ValueError("bias must be bf16 [N]")
+    for g, name in ((norm_q, "norm_q"), (norm_k, "norm_k")):
+        if g is not None and (g.dtype != torch.bfloat16 or g.numel() != 128 or not g.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 [128]")
+    for tb, name in ((rope_cos, "rope_cos"), (rope_sin, "rope_sin")):
+        if tb is not None and (tb.dtype != torch.float32 or tuple(tb.shape) != (M, 64)
+                               or not tb.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous float32 [M, 64]")
+    f = N.NVFP4_G16
+    _need(a_codes, lib.svdq_codes_bytes(f, M, K), "a_codes")
+    _need(a_scales, lib.svdq_scales_bytes(f, M, K), "a_scales")
+    _need(w_codes, lib.svdq_codes_bytes(f, N_, K), "w_codes")
+    _need(w_scales, lib.svdq_scales_bytes(f, N_, K), "w_scales")
+    N.check(lib.svdq_w4a4_linear_qkv_norm_rope(
+        M, N_, K, r, _ptr(a_codes), _ptr(a_scales), _ptr(xl1) if r else None, _ptr(w_codes),
+        _ptr(w_scales), _ptr(L2) if r else None, _ptr(bias), _ptr(norm_q), _ptr(norm_k),
+        float(eps), _ptr(rope_cos), _ptr(rope_sin), _ptr(Y), Y.shape[1], out, _stream(stream)),
+        "svdq_w4a4_linear_qkv_norm_rope")
+    return Y
+
+
 def svdq_tensor_scale(X: torch.Tensor, smooth_inv: torch.Tensor | None = None,
                       scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Two-level NVFP4: float32 [2] = (s_t, RN32(1 / s_t)) of x_hat = RN32(X * smooth_inv)."""

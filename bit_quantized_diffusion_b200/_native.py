@@ -25,7 +25,7 @@ EXPORTS = (
     "awq_w4a16_linear", "svdq_pack", "svdq_unpack", "svdq_check_device_status",
     "svdq_debug_wait_timeout", "svdq_pack_lowrank", "svdq_xl1_splits",
     "svdq_quantize_act_noalloc", "svdq_tensor_scale", "svdq_quantize_act_two_level",
-    "svdq_w4a4_linear_two_level",
+    "svdq_w4a4_linear_two_level", "svdq_w4a4_linear_qkv_norm_rope",
 )
 
 _lib = None
@@ -65,6 +65,8 @@ def load() -> ctypes.CDLL:
         "svdq_quantize_act_two_level": (_I, [_I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
         "svdq_w4a4_linear_two_level": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _I, _I, _P]),
+        "svdq_w4a4_linear_qkv_norm_rope": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                ctypes.c_float, _P, _P, _P, _I, _I, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

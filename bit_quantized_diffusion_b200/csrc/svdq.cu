@@ -118,7 +118,13 @@ svdq_status device_setup(DeviceInfo** out) {
                              static_cast<int>(GmCfg<false>::kSmemBytes)) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(GmCfg<true>::kSmemBytes)) != cudaSuccess)
+                             static_cast<int>(GmCfg<true>::kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(GmCfg<false, true>::kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_nvfp4_gemm_kernel<true, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(GmCfg<true, true>::kSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
@@ -131,6 +137,8 @@ svdq_status device_setup(DeviceInfo** out) {
                           reinterpret_cast<const void*>(quantize_act_kernel<1>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<false>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true>),
+                          reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<false, true>),
+                          reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true, true>),
                           reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<false>),
                           reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<true>),
                           reinterpret_cast<const void*>(awq_gemv_kernel<1>),
@@ -459,11 +467,21 @@ svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, c
 
 namespace {
 
+// the fused QKV epilogue's arguments (svdq_w4a4_linear_qkv_norm_rope)
+struct QkNormArgs {
+  int q_heads;
+  float eps;
+  const void* norm_q;
+  const void* norm_k;
+  const float* rope_cos;
+  const float* rope_sin;
+};
+
 svdq_status w4a4_linear_impl(svdq_format format, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
                              const void* w_scales, const void* L2, const void* bias, void* Y,
                              int ldy, svdq_out out, svdq_stream_t stream, const float* a_tscale,
-                             const float* w_tscale) {
+                             const float* w_tscale, const QkNormArgs* qk = nullptr) {
   if (format != SVDQ_NVFP4_G16 && format != SVDQ_INT4_G64) return SVDQ_ERR_INVALID_ARG;
   if ((a_tscale != nullptr) != (w_tscale != nullptr)) return SVDQ_ERR_INVALID_ARG;
   if (a_tscale != nullptr && format != SVDQ_NVFP4_G16) return SVDQ_ERR_INVALID_ARG;
@@ -480,6 +498,7 @@ svdq_status w4a4_linear_impl(svdq_format format, int M, int N, int K, int r, con
       !aligned16(Y) || (xl1 && !aligned16(xl1)) || (L2 && !aligned16(L2)) ||
       (bias && !aligned16(bias)) || (static_cast<size_t>(ldy) * esz) % 16)
     return SVDQ_ERR_ALIGNMENT;
+  if (qk != nullptr && format != SVDQ_NVFP4_G16) return SVDQ_ERR_UNSUPPORTED;
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
   if (format == SVDQ_INT4_G64)
@@ -533,18 +552,32 @@ svdq_status w4a4_linear_impl(svdq_format format, int M, int N, int K, int r, con
   p.w_tscale = w_tscale;
   p.out_f32 = f32;
   p.status = d->status;
+  p.q_heads = qk != nullptr ? qk->q_heads : 0;
+  p.eps = qk != nullptr ? qk->eps : 0.0f;
+  p.norm_q = qk != nullptr ? static_cast<const __nv_bfloat16*>(qk->norm_q) : nullptr;
+  p.norm_k = qk != nullptr ? static_cast<const __nv_bfloat16*>(qk->norm_k) : nullptr;
+  p.rope_cos = qk != nullptr ? qk->rope_cos : nullptr;
+  p.rope_sin = qk != nullptr ? qk->rope_sin : nullptr;
   p.tiles_m = (M + kGmBM * ctas - 1) / (kGmBM * ctas);
   p.tiles = p.tiles_m * ((N + kGmBN - 1) / kGmBN);
   const int max_units = pair ? d->gemm_pairs : d->num_sms;
   const int units = p.tiles < max_units ? p.tiles : max_units;
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      pair ? launch_kernel(d, w4a4_nvfp4_gemm_kernel<true>, dim3(units * 2), dim3(kGmThreads),
-                           GmCfg<true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
-                           tm_y, p)
-           : launch_kernel(d, w4a4_nvfp4_gemm_kernel<false>, dim3(units), dim3(kGmThreads),
-                           GmCfg<false>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
-                           tm_y, p);
+  cudaError_t e;
+  if (qk != nullptr)
+    e = pair ? launch_kernel(d, w4a4_nvfp4_gemm_kernel<true, true>, dim3(units * 2), dim3(kGmThreads),
+                             GmCfg<true, true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2,
+                             tm_xl1, tm_y, p)
+             : launch_kernel(d, w4a4_nvfp4_gemm_kernel<false, true>, dim3(units), dim3(kGmThreads),
+                             GmCfg<false, true>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2,
+                             tm_xl1, tm_y, p);
+  else
+    e = pair ? launch_kernel(d, w4a4_nvfp4_gemm_kernel<true>, dim3(units * 2), dim3(kGmThreads),
+                             GmCfg<true>::kSmemBytes, cs, 2, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
+                             tm_y, p)
+             : launch_kernel(d, w4a4_nvfp4_gemm_kernel<false>, dim3(units), dim3(kGmThreads),
+                             GmCfg<false>::kSmemBytes, cs, 1, tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1,
+                             tm_y, p);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
@@ -572,6 +605,22 @@ svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a
   if (a_tensor_scale == nullptr || w_tensor_scale == nullptr) return SVDQ_ERR_INVALID_ARG;
   return w4a4_linear_impl(SVDQ_NVFP4_G16, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales,
                           L2, bias, Y, ldy, out, stream, a_tensor_scale, w_tensor_scale);
+}
+
+svdq_status svdq_w4a4_linear_qkv_norm_rope(int M, int N, int K, int r, const void* a_codes,
+                                           const void* a_scales, const float* xl1,
+                                           const void* w_codes, const void* w_scales, const void* L2,
+                                           const void* bias, const void* norm_q, const void* norm_k,
+                                           float eps, const float* rope_cos, const float* rope_sin,
+                                           void* Y, int ldy, svdq_out out, svdq_stream_t stream) {
+  if (N < 384 || N % 384 || !(eps >= 0.0f) || eps > 3.0e38f) return SVDQ_ERR_INVALID_ARG;
+  if ((rope_cos != nullptr) != (rope_sin != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if ((rope_cos && (!aligned16(rope_cos) || !aligned16(rope_sin))) ||
+      (reinterpret_cast<uintptr_t>(norm_q) & 1u) || (reinterpret_cast<uintptr_t>(norm_k) & 1u))
+    return SVDQ_ERR_ALIGNMENT;
+  const QkNormArgs qk{N / 384, eps, norm_q, norm_k, rope_cos, rope_sin};
+  return w4a4_linear_impl(SVDQ_NVFP4_G16, M, N, K, r, a_codes, a_scales, xl1, w_codes, w_scales,
+                          L2, bias, Y, ldy, out, stream, nullptr, nullptr, &qk);
 }
 
 svdq_status svdq_tensor_scale(int M, int K, const void* X, int ldx, const float* smooth_inv,

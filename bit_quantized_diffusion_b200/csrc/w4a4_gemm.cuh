@@ -48,6 +48,18 @@
 // ([0, 256) and [160, 416)), the two scale buffers in [416, 512). The epilogue
 // drains the overlapped columns of a tile first and releases them, so the next
 // tile's MMAs start while the rest of the tile is still being stored.
+//
+// Fused QKV epilogue (kQkNorm; Diffusers blog, the fused QKV section: one to_qkv
+// linear whose output is Q, then K, then V, each head of Q and K normalised by
+// norm_q / norm_k and then rotated by the rotary embedding, in one fused call).
+// Heads are 128 columns, so a 256-column tile holds two whole heads. Each row's
+// head is split between the quadrant's two epilogue warps: each warp sums the
+// squares of its columns of each head (y = alpha acc + bias in float32), the two
+// trade their partial sums through shared memory behind a per-quadrant
+// mbarrier, and each then scales its columns by rsqrt(mean + eps) and the head's
+// weight and turns adjacent pairs (2i, 2i+1) by the row's angle i. Overlapped
+// sub-tiles are released after their first load as usual and kept in registers;
+// the others are read from tensor memory twice. V heads take the plain path.
 #pragma once
 
 #include "sm100.cuh"
@@ -71,7 +83,7 @@ constexpr uint32_t kTmAcc1 = 160, kTmOverlap = 96, kTmSf = 416, kTmSfBuf = 48, k
 static_assert(kTmAcc1 + 256 <= kTmSf && kTmSf + 2 * kTmSfBuf <= kTmCols, "tensor-memory layout");
 static_assert(256 - kTmOverlap == kTmAcc1, "the accumulators overlap by kTmOverlap columns");
 
-template <bool kPair>
+template <bool kPair, bool kQkNorm = false>
 struct GmCfg {
   static constexpr int kCtas = kPair ? 2 : 1;
   static constexpr int kBRows = kGmBN / kCtas;                // B rows staged per CTA
@@ -84,7 +96,15 @@ struct GmCfg {
   static constexpr uint32_t kBars = kBias + kGmEpiWarps * 128 * 4;
   // full, empty, ready, sf landed per stage; acc full, acc free; sf full, sf free per buffer
   static constexpr uint32_t kTmemSlot = kBars + 8 * (4 * kStages + 2 + 2 * 2);
-  static constexpr size_t kSmemBytes = kTmemSlot + 16 + 1024;
+  // fused QKV epilogue only: head weights per epilogue warp [4][32] float32, the
+  // partial sums of squares [2 phases][4 quadrants][2 warps][2 heads][32 rows],
+  // one exchange barrier per quadrant, and a 32 x 32 float32 sub-tile parked by
+  // each of the first half's four epilogue warps
+  static constexpr uint32_t kGamma = kTmemSlot + 16;
+  static constexpr uint32_t kRed = kGamma + kGmEpiWarps * 128 * 4;
+  static constexpr uint32_t kNormBars = kRed + 2 * 4 * 2 * 2 * 32 * 4;
+  static constexpr uint32_t kPark = kNormBars + 4 * 8;
+  static constexpr size_t kSmemBytes = (kQkNorm ? kPark + 4 * 4096 : kTmemSlot + 16) + 1024;
   static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
   static_assert(kLrBTile + 2 * kGmLrATile <= kStageBytes, "a low-rank slot fits in a stage");
 };
@@ -99,9 +119,18 @@ struct GemmParams {
   const float* w_tscale;
   int out_f32;
   uint32_t* status;
+  // fused QKV epilogue (kQkNorm): q_heads heads of 128 columns each of Q and K
+  // (columns [0, 128 q_heads) and [128 q_heads, 256 q_heads)); head weights
+  // [128] bf16 or null (1); rotation tables cos, sin [M, 64] float32 or null
+  int q_heads;
+  float eps;
+  const __nv_bfloat16* norm_q;
+  const __nv_bfloat16* norm_k;
+  const float* rope_cos;
+  const float* rope_sin;
 };
 
-template <bool kPair>
+template <bool kPair, bool kQkNorm = false>
 __global__ void __launch_bounds__(kGmThreads, 1)
     w4a4_nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                            const __grid_constant__ CUtensorMap tm_b,
@@ -110,7 +139,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                            const __grid_constant__ CUtensorMap tm_l2,
                            const __grid_constant__ CUtensorMap tm_xl1,
                            const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
-  using Cfg = GmCfg<kPair>;
+  using Cfg = GmCfg<kPair, kQkNorm>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,6 +193,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       mbar_init(bar_sf_full(b), 4 * Cfg::kCtas);  // quadrant warps of the pair
       mbar_init(bar_sf_free(b), 1);               // MMA commit
     }
+    if constexpr (kQkNorm)
+      for (int q = 0; q < 4; ++q) mbar_init(sbase + Cfg::kNormBars + 8 * q, 2);  // a quadrant's two epilogue warps
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
@@ -454,6 +485,60 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     bool ok = true;
     int stores = 0;
     const float alpha = p.a_tscale != nullptr ? __fmul_rn(p.a_tscale[0], p.w_tscale[0]) : 1.0f;
+    // stage the warp's 32 x 32 sub-tile (its rows, columns n0 + j0 ..) in the TMA
+    // store's swizzled layout and store it
+    auto store_sub = [&](const float (&y)[32], int n0, int j0, int mrow) {
+      uint32_t buf;
+      if (p.out_f32) {
+        buf = out_buf;  // one 4 KB buffer, rows of 128 B, 128-byte swizzle
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           buf + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                       "f"(y[4 * c]), "f"(y[4 * c + 1]), "f"(y[4 * c + 2]), "f"(y[4 * c + 3])
+                       : "memory");
+      } else {
+        buf = out_buf + (stores & 1) * 2048;  // two 2 KB buffers, rows of 64 B, 64-byte swizzle
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+          pk[j] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)),
+                       "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                       : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tm_y, buf, n0 + j0, mrow + quad * 32);
+        bulk_commit();
+      }
+      ++stores;
+    };
+    // y = alpha * acc + bias for one sub-tile, one rounding (alpha = 1 without
+    // tensor scales: the plain sum); with two-level scales the accumulator holds
+    // the 4-bit product and the low-rank term divided by alpha
+    auto finish = [&](const uint32_t (&acc)[32], int t, float (&y)[32]) {
+      const float4* bv = reinterpret_cast<const float4*>(bias_s + t * 32);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 b = bv[q4];
+        y[4 * q4 + 0] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 0]), alpha, b.x);
+        y[4 * q4 + 1] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 1]), alpha, b.y);
+        y[4 * q4 + 2] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 2]), alpha, b.z);
+        y[4 * q4 + 3] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 3]), alpha, b.w);
+      }
+    };
+    int nt = 0;  // fused-norm tiles so far: the phase of this quadrant's exchange barrier
     for (int i = 0; i < my_tiles && ok; ++i) {
       int m0, n0;
       tile_mn(i, m0, n0);
@@ -476,17 +561,164 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         sub_col[2] = other0 + 96;
         sub_col[3] = other0 + 128;
       }
-      // bias for this warp's sub-tiles, fetched before the accumulator is ready
+      const bool norm_tile = kQkNorm && n0 < 256 * p.q_heads;  // holds a Q or K head
+      // bias (and head weights) for this warp's sub-tiles, fetched before the
+      // accumulator is ready
       __syncwarp();
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int n = n0 + sub_col[t] + lane;
         bias_s[t * 32 + lane] = (p.bias != nullptr && n < p.N) ? __bfloat162float(p.bias[n]) : 0.0f;
       }
+      if constexpr (kQkNorm) {
+        if (norm_tile) {
+          float* gamma_s = reinterpret_cast<float*>(smem + Cfg::kGamma) + (warp - 6) * 128;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int g = n0 / 128 + (sub_col[t] >> 7);  // global head
+            const __nv_bfloat16* w =
+                g < p.q_heads ? p.norm_q : (g < 2 * p.q_heads ? p.norm_k : nullptr);
+            gamma_s[t * 32 + lane] = w != nullptr ? __bfloat162float(w[(sub_col[t] & 127) + lane]) : 1.0f;
+          }
+        }
+      }
       __syncwarp();
       ok = mbar_wait(bar_acc_full, i & 1, p.status);
       if (!ok) break;
       tc_fence_after();
+      if constexpr (kQkNorm) {
+        if (norm_tile) {
+          // The overlapped sub-tiles are released once read: the first stays in
+          // registers, the first half's second is parked, as y, in shared memory.
+          uint32_t h0[32];
+          const uint32_t park = sbase + Cfg::kPark + quad * 4096;  // first-half warps only
+          float ss0 = 0.0f, ss1 = 0.0f;  // the row's sums of squares over this warp's columns of either head
+          auto add_sq = [&](const float (&y)[32], int t) {
+            float sq = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) sq = __fmaf_rn(y[q], y[q], sq);
+            if (sub_col[t] < 128) ss0 += sq;
+            else ss1 += sq;
+          };
+          if (half == 0) {
+            // the second overlapped sub-tile first: to y, into the sums, parked
+            uint32_t h1[32];
+            tmem_ld32(t_row + sub_col[1], h1);
+            tmem_ld_wait();
+            if (mrow < p.M) {
+              float y[32];
+              finish(h1, 1, y);
+              add_sq(y, 1);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                 park + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                             "f"(y[4 * c]), "f"(y[4 * c + 1]), "f"(y[4 * c + 2]), "f"(y[4 * c + 3])
+                             : "memory");
+            }
+          }
+          tmem_ld32(t_row + sub_col[0], h0);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (kPair) mbar_arrive_remote(free_bar);
+            else mbar_arrive(free_bar);
+          }
+          if (mrow >= p.M) continue;  // the same for both warps of the quadrant
+          // pass 1: the rest of the sums of squares
+          {
+            float y[32];
+            finish(h0, 0, y);
+            add_sq(y, 0);
+          }
+#pragma unroll
+          for (int t = 1; t < 4; ++t) {
+            if (t == 1 && half == 0) continue;
+            uint32_t acc[32];
+            tmem_ld32(t_row + sub_col[t], acc);
+            tmem_ld_wait();
+            float y[32];
+            finish(acc, t, y);
+            add_sq(y, t);
+          }
+          // trade the partial sums with the quadrant's other warp (two phases of
+          // slots: a warp can be at most one tile ahead of its partner)
+          float* red = reinterpret_cast<float*>(smem + Cfg::kRed);
+          float* mine = red + (((nt & 1) * 4 + quad) * 2 + half) * 64;
+          const float* theirs = red + (((nt & 1) * 4 + quad) * 2 + (half ^ 1)) * 64;
+          mine[lane] = ss0;
+          mine[32 + lane] = ss1;
+          __syncwarp();
+          const uint32_t xbar = sbase + Cfg::kNormBars + 8 * quad;
+          if (lane == 0) mbar_arrive(xbar);
+          ok = mbar_wait(xbar, nt & 1, p.status);
+          ++nt;
+          if (!ok) break;
+          const float rs0 = rsqrtf(__fmaf_rn(ss0 + theirs[lane], 1.0f / 128.0f, p.eps));
+          const float rs1 = rsqrtf(__fmaf_rn(ss1 + theirs[32 + lane], 1.0f / 128.0f, p.eps));
+          // pass 2: scale, weight, rotate, store. src 0: h0; 1: the parked y; 2: tensor memory
+          const float* gamma_s = reinterpret_cast<const float*>(smem + Cfg::kGamma) + (warp - 6) * 128;
+          const int m = mrow + quad * 32 + lane;
+          const size_t trow = static_cast<size_t>(m < p.M ? m : 0) * 64;  // rows past M: any valid row
+          auto emit = [&](int t, int src) {
+            const int j0 = sub_col[t];
+            float y[32];
+            if (src == 0) {
+              finish(h0, t, y);
+            } else if (src == 1) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(y[4 * c]), "=f"(y[4 * c + 1]), "=f"(y[4 * c + 2]), "=f"(y[4 * c + 3])
+                             : "r"(park + lane * 128 + ((c ^ (lane & 7)) << 4))
+                             : "memory");
+            } else {
+              uint32_t acc[32];
+              tmem_ld32(t_row + j0, acc);
+              tmem_ld_wait();
+              finish(acc, t, y);
+            }
+            if (n0 / 128 + (j0 >> 7) < 2 * p.q_heads) {
+              const float rs = j0 < 128 ? rs0 : rs1;
+              const float4* gv = reinterpret_cast<const float4*>(gamma_s + t * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 w = gv[q4];
+                y[4 * q4 + 0] = __fmul_rn(__fmul_rn(y[4 * q4 + 0], rs), w.x);
+                y[4 * q4 + 1] = __fmul_rn(__fmul_rn(y[4 * q4 + 1], rs), w.y);
+                y[4 * q4 + 2] = __fmul_rn(__fmul_rn(y[4 * q4 + 2], rs), w.z);
+                y[4 * q4 + 3] = __fmul_rn(__fmul_rn(y[4 * q4 + 3], rs), w.w);
+              }
+              if (p.rope_cos != nullptr) {
+                // the sub-tile's 16 pairs are angles (j0 mod 128) / 2 .. + 15 of the row
+                const float4* cp = reinterpret_cast<const float4*>(p.rope_cos + trow + ((j0 & 127) >> 1));
+                const float4* sp = reinterpret_cast<const float4*>(p.rope_sin + trow + ((j0 & 127) >> 1));
+                auto turn = [](float& a, float& b, float c, float sn) {
+                  const float x = a, z = b;
+                  a = __fmaf_rn(x, c, -__fmul_rn(z, sn));
+                  b = __fmaf_rn(z, c, __fmul_rn(x, sn));
+                };
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const float4 c = __ldg(cp + q4), sn = __ldg(sp + q4);
+                  turn(y[8 * q4 + 0], y[8 * q4 + 1], c.x, sn.x);
+                  turn(y[8 * q4 + 2], y[8 * q4 + 3], c.y, sn.y);
+                  turn(y[8 * q4 + 4], y[8 * q4 + 5], c.z, sn.z);
+                  turn(y[8 * q4 + 6], y[8 * q4 + 7], c.w, sn.w);
+                }
+              }
+            }
+            if (n0 + j0 >= p.N) return;
+            store_sub(y, n0, j0, mrow);
+          };
+          emit(0, 0);
+          emit(1, half == 0 ? 1 : 2);
+          emit(2, 2);
+          emit(3, 2);
+          continue;
+        }
+      }
       uint32_t acc_next[32];  // the first half's second overlapped sub-tile
       for (int t = 0; t < 4; ++t) {
         const int j0 = sub_col[t];
@@ -510,54 +742,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
         if (n0 + j0 >= p.N || mrow >= p.M) continue;  // warp-uniform
         float y[32];
-        const float4* bv = reinterpret_cast<const float4*>(bias_s + t * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          // y = alpha * acc + bias, one rounding (alpha = 1 without tensor scales: the
-          // plain sum); with two-level scales the accumulator holds the 4-bit product
-          // and the low-rank term divided by alpha
-          const float4 b = bv[q4];
-          y[4 * q4 + 0] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 0]), alpha, b.x);
-          y[4 * q4 + 1] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 1]), alpha, b.y);
-          y[4 * q4 + 2] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 2]), alpha, b.z);
-          y[4 * q4 + 3] = __fmaf_rn(__uint_as_float(acc[4 * q4 + 3]), alpha, b.w);
-        }
-        // stage the warp's 32 x 32 sub-tile in the TMA store's swizzled layout
-        uint32_t buf;
-        if (p.out_f32) {
-          buf = out_buf;  // one 4 KB buffer, rows of 128 B, 128-byte swizzle
-          if (lane == 0) bulk_wait_read<0>();
-          __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             buf + lane * 128 + ((c ^ (lane & 7)) << 4)),
-                         "f"(y[4 * c]), "f"(y[4 * c + 1]), "f"(y[4 * c + 2]), "f"(y[4 * c + 3])
-                         : "memory");
-        } else {
-          buf = out_buf + (stores & 1) * 2048;  // two 2 KB buffers, rows of 64 B, 64-byte swizzle
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
-            pk[j] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)),
-                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                         : "memory");
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, buf, n0 + j0, mrow + quad * 32);
-          bulk_commit();
-        }
-        ++stores;
+        finish(acc, t, y);
+        store_sub(y, n0, j0, mrow);
       }
     }
     if (lane == 0) bulk_wait_all();

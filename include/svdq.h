@@ -227,6 +227,36 @@ svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a
                                        void* Y, int ldy, svdq_out out, svdq_stream_t stream);
 
 /*
+ * svdq_w4a4_linear_qkv_norm_rope -- the fused QKV projection of an attention
+ * block with its head normalisation and rotary embedding in the GEMM's epilogue
+ * (Diffusers blog, the fused QKV section: to_q, to_k, to_v joined along the
+ * output dimension in the order Q, K, V into one SVDQ linear, whose output goes
+ * through norm_q / norm_k per head and then the rotary embedding in one fused
+ * call). svdq_w4a4_linear in NVFP4, then on each row m of Y:
+ *   heads of 128 columns, H = N / 384 of each of Q (columns [0, 128 H)), K
+ *   ([128 H, 256 H)) and V ([256 H, 384 H));
+ *   each head v of Q and K: z = v * rsqrt(mean(v^2) + eps) * gamma, gamma the
+ *   head weight (norm_q for Q, norm_k for K); then each pair (z[2i], z[2i+1]) ->
+ *   (z[2i] cos - z[2i+1] sin, z[2i+1] cos + z[2i] sin), cos = rope_cos[m][i] and
+ *   sin = rope_sin[m][i];
+ *   V as svdq_w4a4_linear computes it.
+ * All of it in float32 from the accumulator, with one rounding at the output.
+ *   N        multiple of 384 (three projections of whole 128-column heads)
+ *   norm_q, norm_k  device bf16 [128], 2-byte aligned, or NULL (weight 1)
+ *   eps      finite, >= 0 (a head whose values are all zero needs eps > 0)
+ *   rope_cos, rope_sin  device float32 [M, 64] row-major (row m: the angles of
+ *            token row m), 16-byte aligned; both NULL: no rotation
+ * Other arguments, layouts and errors as for svdq_w4a4_linear; INVALID_ARG when
+ * N is not a multiple of 384, eps is out of range or only one table is given.
+ */
+svdq_status svdq_w4a4_linear_qkv_norm_rope(int M, int N, int K, int r, const void* a_codes,
+                                           const void* a_scales, const float* xl1,
+                                           const void* w_codes, const void* w_scales, const void* L2,
+                                           const void* bias, const void* norm_q, const void* norm_k,
+                                           float eps, const float* rope_cos, const float* rope_sin,
+                                           void* Y, int ldy, svdq_out out, svdq_stream_t stream);
+
+/*
  * awq_w4a16_linear -- step a7, the AWQ W4A16 linear for small-M modulation
  * projections (Diffusers blog, "From SVDQuant to Nunchaku Lite": awq_w4a16 for
  * the memory-bound adaptive-norm projections).

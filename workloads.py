@@ -148,3 +148,22 @@ def custom_svdq(name: str, M: int, K: int, N: int, r: int, fmt: str = "nvfp4",
     """A small workload of the same structure, for tests that need ragged sizes."""
     return SvdqShape(name, M, K, N, r, fmt, n_outliers, outlier_scale, spike_rank,
                      spike_sv, bias, seed)
+
+
+def qkv_epilogue_inputs(M: int, seed: int, angles: str = "uniform") -> dict:
+    """Inputs of the fused QKV epilogue: head weights gamma_q, gamma_k [128] as
+    bfloat16 bits (~ 1 + N(0, 0.1), the spread of trained RMS-norm weights), and
+    rotation tables cos, sin [M, 64] float32. ``angles`` "uniform" draws every
+    angle from U(-pi, pi); "positions" takes row m as token position m with pair
+    i at frequency 10000^(-i/64), the usual rotary layout of one position axis."""
+    rng = np.random.default_rng(seed)
+    gq = to_bf16_bits(1.0 + rng.standard_normal(128) * 0.1)
+    gk = to_bf16_bits(1.0 + rng.standard_normal(128) * 0.1)
+    if angles == "uniform":
+        th = rng.uniform(-np.pi, np.pi, (M, 64))
+    elif angles == "positions":
+        th = np.arange(M, dtype=np.float64)[:, None] * 10000.0 ** (-np.arange(64) / 64.0)[None, :]
+    else:
+        raise ValueError(angles)
+    return {"norm_q": gq, "norm_k": gk, "cos": np.cos(th).astype(np.float32),
+            "sin": np.sin(th).astype(np.float32)}
