@@ -8,8 +8,8 @@ from __future__ import annotations
 import torch
 
 from . import (awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_quantize_act_two_level,
-               svdq_scales_bytes, svdq_tensor_scale, svdq_w4a4_linear, svdq_w4a4_linear_two_level,
-               svdq_xl1_splits)
+               svdq_scales_bytes, svdq_tensor_scale, svdq_w4a4_linear, svdq_w4a4_linear_qkv_norm_rope,
+               svdq_w4a4_linear_two_level, svdq_xl1_splits)
 
 
 class SvdqW4A4Linear:
@@ -59,6 +59,44 @@ class SvdqW4A4Linear:
                                                stream=stream)
         return svdq_w4a4_linear(codes, scales, xl1, self.w["w_codes"], self.w["w_scales"], self.w["L2"],
                                 self.bias, M, self.N, self.K, fmt=self.fmt, Y=y, stream=stream)
+
+    __call__ = forward
+
+
+class SvdqQkvNormRope(SvdqW4A4Linear):
+    """The fused QKV projection of an attention block (Diffusers blog, the fused QKV
+    section: to_q, to_k, to_v joined into one SVDQ linear, followed by norm_q / norm_k
+    per head and the rotary embedding in one fused call). Weights prepared for the
+    joined [3 H 128, K] projection, NVFP4, one-level; norm_q, norm_k bf16 [128] or None.
+    forward(x, rope_cos, rope_sin) takes the rows' angle tables, float32 [M, 64] each
+    (or None: no rotation), and returns Q | K | V [M, 3 H 128], Q and K normalised and
+    rotated."""
+
+    def __init__(self, weights: dict, bias: torch.Tensor | None, max_tokens: int,
+                 norm_q: torch.Tensor | None = None, norm_k: torch.Tensor | None = None,
+                 eps: float = 1e-6):
+        if weights["fmt"] != "nvfp4" or weights.get("w_tscale") is not None:
+            raise ValueError("the fused QKV projection takes one-level NVFP4 weights")
+        if weights["N"] % 384:
+            raise ValueError(f"N = {weights['N']} is not Q, K, V of whole 128-column heads")
+        super().__init__(weights, bias, max_tokens)
+        self.norm_q, self.norm_k, self.eps = norm_q, norm_k, float(eps)
+        self.heads = weights["N"] // 384
+
+    def forward(self, x: torch.Tensor, rope_cos: torch.Tensor | None = None,
+                rope_sin: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+        M = x.shape[0]
+        if M > self.max_tokens:
+            raise ValueError(f"{M} tokens > workspace for {self.max_tokens}")
+        xl1 = self.xl1[:svdq_xl1_splits(M, self.K, self.r) * M * self.r] if self.r else None
+        codes, scales, xl1 = svdq_quantize_act(x, self.w["L1s"], self.w["smooth_inv"], fmt="nvfp4",
+                                               codes=self.codes, scales=self.scales, xl1=xl1,
+                                               stream=stream)
+        return svdq_w4a4_linear_qkv_norm_rope(codes, scales, xl1, self.w["w_codes"], self.w["w_scales"],
+                                              self.w["L2"], self.bias, self.norm_q, self.norm_k,
+                                              rope_cos, rope_sin, M, self.N, self.K, eps=self.eps, Y=y,
+                                              stream=stream)
 
     __call__ = forward
 

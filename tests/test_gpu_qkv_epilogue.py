@@ -144,3 +144,31 @@ def test_full_size_flux_qkv(bq):
                           F.bf16_from_bits(ep["norm_k"]), 1e-6, ep["cos"][rows], ep["sin"][rows])
     C.assert_gemm_close(as_f64(y[rows])[:, :2 * H * D], ref[:, :2 * H * D], bf16_out=True,
                         what="Q, K (full size)")
+
+
+def test_layer_class_matches_the_oracle(bq):
+    """SvdqQkvNormRope on oracle-prepared weights (one call per forward after the
+    quantizer), against the oracle's layer followed by its epilogue."""
+    from bit_quantized_diffusion_b200.layers import SvdqQkvNormRope
+    M, H, K, r = 384, 2, 1024, 32
+    shape = WL.custom_svdq("qkv_layer", M, K, 3 * H * D, r, seed=91, n_outliers=8,
+                           outlier_scale=50.0, spike_rank=8, spike_sv=5.0)
+    layer = C.oracle_layer(shape)
+    ep = WL.qkv_epilogue_inputs(M, seed=92)
+    si = C.f32_tensor(layer["smooth_inv"])
+    w = {"smooth_inv": si, "L1s": bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(layer["L1"])), si),
+         "L2": C.bf16_tensor(F.bf16_bits(layer["L2"])),
+         "w_codes": C.u8_tensor(C.tiled_codes("nvfp4", layer["w_codes"])),
+         "w_scales": C.u8_tensor(C.tiled_scales("nvfp4", layer["w_scales"])),
+         "fmt": "nvfp4", "N": shape.N, "K": K, "r": r}
+    mod = SvdqQkvNormRope(w, C.bf16_tensor(layer["bias_bits"]), max_tokens=512,
+                          norm_q=C.bf16_tensor(ep["norm_q"]), norm_k=C.bf16_tensor(ep["norm_k"]))
+    y = mod(C.bf16_tensor(layer["x_bits"]), C.f32_tensor(ep["cos"]), C.f32_tensor(ep["sin"]))
+    assert bq.svdq_check_device_status() == 0
+    fwd = S.svdq_forward("nvfp4", layer["x_bits"], layer["smooth_inv"], layer["L1"], layer["L2"],
+                         layer["w_codes"], layer["w_scales"], layer["bias_bits"])
+    ref = E.qkv_norm_rope(fwd["Y"], H, F.bf16_from_bits(ep["norm_q"]), F.bf16_from_bits(ep["norm_k"]),
+                          1e-6, ep["cos"], ep["sin"])
+    got = as_f64(y)
+    C.assert_gemm_close(got[:, :2 * H * D], ref[:, :2 * H * D], bf16_out=True, what="Q, K (layer)")
+    C.assert_gemm_close(got[:, 2 * H * D:], ref[:, 2 * H * D:], bf16_out=True, what="V (layer)")
