@@ -19,6 +19,13 @@ records events only at step boundaries, and the per-kernel times (and the
 roofline of the GEMM) come from a second pass of the same steps with an event
 between every two kernels.
 
+Beside the step, and not part of it, two variants of the same layer are timed
+call by call after the flush: two-level NVFP4 (svdq_tensor_scale,
+svdq_quantize_act_two_level, svdq_w4a4_linear_two_level) and the fused QKV
+projection (svdq_w4a4_linear_qkv_norm_rope: the layer's 9216 columns as 24 heads
+each of Q, K, V, with the heads of Q and K RMS-normalised and rotated in the
+GEMM's epilogue). They appear under "kernels".
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 With N > 1 (torchrun, one process per GPU) every rank runs the same layer on

@@ -11,6 +11,15 @@
  * "quantization_config": svdq_w4a4 {precision, group_size, rank} and awq_w4a16
  * {precision int4, group_size 64}.
  *
+ * Calls: the activation quantizer with the fused down-projection
+ * (svdq_quantize_act, svdq_quantize_act_noalloc), the 4-bit GEMM with the fused
+ * up-projection (svdq_w4a4_linear), NVFP4 with a per-tensor second scale level
+ * (svdq_tensor_scale, svdq_quantize_act_two_level, svdq_w4a4_linear_two_level),
+ * the fused QKV projection with head norm and rotation
+ * (svdq_w4a4_linear_qkv_norm_rope), the AWQ W4A16 linear (awq_w4a16_linear),
+ * layout conversion (svdq_pack, svdq_unpack, svdq_pack_lowrank), buffer sizes,
+ * and the device status word (svdq_check_device_status).
+ *
  * Conventions for every call:
  *  - Memory: the caller allocates and owns every buffer. Pointers named as device
  *    pointers must be device memory, 16-byte aligned. The library allocates
