@@ -7,6 +7,7 @@ from __future__ import annotations
 
 import torch
 
+from . import prep
 from . import (awq_w4a16_linear, svdq_codes_bytes, svdq_quantize_act, svdq_quantize_act_two_level,
                svdq_scales_bytes, svdq_tensor_scale, svdq_w4a4_linear, svdq_w4a4_linear_qkv_norm_rope,
                svdq_w4a4_linear_two_level, svdq_xl1_splits)
@@ -38,6 +39,16 @@ class SvdqW4A4Linear:
         # the down-projection's partial sums: at most 8 splits of max_tokens rows
         self.xl1 = (torch.empty(8 * max_tokens * self.r, dtype=torch.float32, device=dev)
                     if self.r else None)
+
+    @classmethod
+    def from_linear(cls, weight: torch.Tensor, bias: torch.Tensor | None, x_absmax: torch.Tensor,
+                    rank: int, max_tokens: int, fmt: str = "nvfp4", two_level: bool = False,
+                    act_scale: torch.Tensor | None = None):
+        """From an nn.Linear's weight [N, K] bf16 (and bias [N] bf16 or None) and the
+        calibration activations' per-channel max |X| [K]: smoothing, SVD split and the
+        residual quantized by the library (prep.prepare_svdq_weights)."""
+        w = prep.prepare_svdq_weights(weight, x_absmax, rank, fmt, two_level=two_level)
+        return cls(w, bias, max_tokens, act_scale=act_scale)
 
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         M = x.shape[0]
@@ -83,6 +94,32 @@ class SvdqQkvNormRope(SvdqW4A4Linear):
         self.norm_q, self.norm_k, self.eps = norm_q, norm_k, float(eps)
         self.heads = weights["N"] // 384
 
+    @classmethod
+    def from_linears(cls, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                     biases: tuple | None, x_absmax: torch.Tensor, rank: int, max_tokens: int,
+                     norm_q: torch.Tensor | None = None, norm_k: torch.Tensor | None = None,
+                     eps: float = 1e-6):
+        """From the to_q, to_k, to_v weights [H 128, K] bf16 (biases: three [H 128] bf16
+        tensors or None each, or None): the three are joined along the output dimension
+        in the order Q, K, V into one [3 H 128, K] projection, which is prepared once
+        (smoothing from x_absmax, SVD split, quantized residual)."""
+        if not (q.shape == k.shape == v.shape) or q.dim() != 2 or q.shape[0] % 128:
+            raise ValueError("to_q, to_k, to_v must be equal [H 128, K] weights")
+        w = torch.cat([q, k, v], dim=0)
+        bias = None
+        if biases is not None and any(b is not None for b in biases):
+            bias = torch.cat([b if b is not None else torch.zeros(q.shape[0], dtype=q.dtype, device=q.device)
+                              for b in biases])
+        return cls.from_linear(w, bias, x_absmax, rank, max_tokens, norm_q=norm_q, norm_k=norm_k, eps=eps)
+
+    @classmethod
+    def from_linear(cls, weight: torch.Tensor, bias: torch.Tensor | None, x_absmax: torch.Tensor,
+                    rank: int, max_tokens: int, norm_q: torch.Tensor | None = None,
+                    norm_k: torch.Tensor | None = None, eps: float = 1e-6):
+        """From an already joined to_qkv weight [3 H 128, K] bf16 (rows Q, then K, then V)."""
+        weights = prep.prepare_svdq_weights(weight, x_absmax, rank, "nvfp4")
+        return cls(weights, bias, max_tokens, norm_q=norm_q, norm_k=norm_k, eps=eps)
+
     def forward(self, x: torch.Tensor, rope_cos: torch.Tensor | None = None,
                 rope_sin: torch.Tensor | None = None, y: torch.Tensor | None = None,
                 stream=None) -> torch.Tensor:
@@ -105,6 +142,12 @@ class AwqW4A16Linear:
     def __init__(self, weights: dict, bias: torch.Tensor | None):
         self.w = weights
         self.bias = bias
+
+    @classmethod
+    def from_linear(cls, weight: torch.Tensor, bias: torch.Tensor | None):
+        """From an nn.Linear's weight [N, K] bf16: asymmetric int4, group 64, packed
+        (prep.prepare_awq_weights)."""
+        return cls(prep.prepare_awq_weights(weight), bias)
 
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         return awq_w4a16_linear(x, self.w["qweight"], self.w["sz"], self.bias, self.w["N"], Y=y,

@@ -106,3 +106,54 @@ def test_one_level_layer(monkeypatch):
     layer(torch.zeros(64, 512, dtype=BF))
     assert [c[0] for c in rec.calls] == ["quantize", "linear"]
     assert rec.calls[0][4] is None  # r = 0: no down-projection
+
+
+def fake_prep(monkeypatch):
+    seen = {}
+
+    def prepare(w, x_absmax, rank, fmt="nvfp4", two_level=False):
+        seen.update(w=w, x_absmax=x_absmax, rank=rank, fmt=fmt, two_level=two_level)
+        N, K = w.shape
+        return weights(N, K, rank, fmt, two_level)
+
+    def prepare_awq(w):
+        seen.update(awq=w)
+        return {"qweight": None, "sz": None, "N": w.shape[0], "K": w.shape[1]}
+
+    monkeypatch.setattr(L.prep, "prepare_svdq_weights", prepare)
+    monkeypatch.setattr(L.prep, "prepare_awq_weights", prepare_awq)
+    return seen
+
+
+def test_from_linears_joins_q_k_v_in_order(monkeypatch):
+    seen = fake_prep(monkeypatch)
+    K, Hd = 512, 2 * 128
+    q, k, v = (torch.full((Hd, K), float(i), dtype=BF) for i in (1, 2, 3))
+    bq_, bv = torch.full((Hd,), 1.0, dtype=BF), torch.full((Hd,), 3.0, dtype=BF)
+    ax = torch.ones(K)
+    gq = torch.ones(128, dtype=BF)
+    layer = L.SvdqQkvNormRope.from_linears(q, k, v, (bq_, None, bv), ax, 32, max_tokens=64,
+                                           norm_q=gq, eps=1e-5)
+    w = seen["w"]
+    assert w.shape == (3 * Hd, K) and seen["rank"] == 32 and seen["x_absmax"] is ax
+    assert torch.equal(w[:Hd], q) and torch.equal(w[Hd:2 * Hd], k) and torch.equal(w[2 * Hd:], v)
+    # a missing bias is zero in its third of the joined bias
+    assert torch.equal(layer.bias[:Hd], bq_) and not layer.bias[Hd:2 * Hd].any()
+    assert torch.equal(layer.bias[2 * Hd:], bv)
+    assert layer.heads == 2 and layer.norm_q is gq and layer.norm_k is None and layer.eps == 1e-5
+    assert L.SvdqQkvNormRope.from_linears(q, k, v, None, ax, 0, max_tokens=8).bias is None
+    with pytest.raises(ValueError):
+        L.SvdqQkvNormRope.from_linears(q, k[:128], v, None, ax, 0, max_tokens=8)
+
+
+def test_from_linear_constructors(monkeypatch):
+    seen = fake_prep(monkeypatch)
+    w = torch.zeros(256, 512, dtype=BF)
+    b = torch.zeros(256, dtype=BF)
+    scale = torch.ones(2)
+    lin = L.SvdqW4A4Linear.from_linear(w, b, torch.ones(512), 16, max_tokens=32, two_level=True,
+                                       act_scale=scale)
+    assert seen["w"] is w and seen["two_level"] and lin.two_level and lin.act_scale is scale
+    assert lin.bias is b and lin.r == 16
+    awq = L.AwqW4A16Linear.from_linear(w, b)
+    assert seen["awq"] is w and awq.bias is b and awq.w["N"] == 256
