@@ -2,6 +2,7 @@
 
 import ml_dtypes
 import numpy as np
+import pytest
 
 import workloads as WL
 
@@ -33,3 +34,19 @@ def test_spike_is_present():
     w = WL.bf16_bits_to_f32(WL.svdq_inputs(shape)["W"]).astype(np.float64)
     s = np.linalg.svd(w, compute_uv=False)
     assert np.all(s[:8] > 4.5) and s[8] < 0.02 * (np.sqrt(192) + np.sqrt(256)) * 1.2
+
+
+def test_qkv_epilogue_inputs():
+    a = WL.qkv_epilogue_inputs(37, seed=3)
+    b = WL.qkv_epilogue_inputs(37, seed=3)
+    assert all(np.array_equal(a[k], b[k]) for k in a)
+    assert a["norm_q"].shape == (128,) and a["norm_q"].dtype == np.uint16
+    assert a["cos"].shape == (37, 64) and a["cos"].dtype == np.float32
+    # each (cos, sin) pair is a unit vector up to float32 rounding
+    assert np.allclose(a["cos"].astype(np.float64) ** 2 + a["sin"].astype(np.float64) ** 2, 1.0, atol=1e-6)
+    # position angles: row 0 is the identity, and pair 0 turns by exactly one radian per row
+    p = WL.qkv_epilogue_inputs(5, seed=0, angles="positions")
+    assert np.array_equal(p["cos"][0], np.ones(64, np.float32)) and not p["sin"][0].any()
+    assert np.allclose(p["cos"][:, 0], np.cos(np.arange(5)), atol=1e-7)
+    with pytest.raises(ValueError):
+        WL.qkv_epilogue_inputs(5, seed=0, angles="random")
