@@ -65,9 +65,9 @@ def prepare_svdq_weights(w: torch.Tensor, x_absmax: torch.Tensor, rank: int,
     else:
         w_tscale = None
         w_codes, w_scales, _ = svdq_quantize_act(R, None, None, fmt=fmt)
-    return {"smooth_inv": smooth_inv.contiguous(), "L1": L1, "L1s": L1s, "L2": L2.contiguous() if L2 is not None else None,
-            "w_codes": w_codes, "w_scales": w_scales, "w_tscale": w_tscale, "R": R, "fmt": fmt, "N": N,
-            "K": K, "r": rank}
+    return {"smooth_inv": smooth_inv.contiguous(), "L1": L1, "L1s": L1s,
+            "L2": L2.contiguous() if L2 is not None else None, "w_codes": w_codes, "w_scales": w_scales,
+            "w_tscale": w_tscale, "R": R, "fmt": fmt, "N": N, "K": K, "r": rank}
 
 
 def prepare_awq_weights(w: torch.Tensor) -> dict:
