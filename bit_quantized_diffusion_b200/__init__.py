@@ -22,12 +22,19 @@ def _fmt(fmt) -> int:
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
+    """A tensor's device address. The library launches on the current device
+    (and its tensor maps and static arrays are that device's), so a tensor on
+    another device is refused here rather than read across devices."""
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{cur}: "
+                         f"call under torch.cuda.device({t.device})")
     return t.data_ptr()
 
 

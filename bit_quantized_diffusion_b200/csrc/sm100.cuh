@@ -153,14 +153,6 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Warm L2 with [src, src + bytes) (16-byte aligned, a multiple of 16 bytes);
-// no data reaches this SM and nothing waits for it.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-               "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int c0, int c1) {
   asm volatile(
@@ -199,11 +191,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
 // outstanding writes.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-// Arrive on an mbarrier given by its shared::cluster address (possibly another CTA's).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 // Plain (non-tensor) bulk copy global -> shared; src, dst 16-byte aligned, bytes % 16 == 0.
@@ -295,41 +282,8 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// int8 x int8 -> s32 MMA.
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// kind::f8f6f4 MMA (8-bit float operands, f32 accumulate); K = 32 per instruction.
-__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Each thread of the warp reads 16 consecutive 32-bit columns of its own lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
 }
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own lane.
@@ -456,22 +410,6 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t M, uint32_t N) {
          | ((M >> 4) << 24);  // M / 16
 }
 
-// Instruction descriptor, kind::i8: signed int8 A/B, s32 accumulator, K-major.
-__host__ __device__ constexpr uint32_t idesc_s8_s32(uint32_t M, uint32_t N) {
-  return (2u << 4)            // D format: s32
-         | (1u << 7)          // A: signed int8
-         | (1u << 10)         // B: signed int8
-         | ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-
-// Instruction descriptor, kind::f8f6f4: E4M3 A and B, f32 accumulator, K-major.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
-  return (1u << 4)            // D format: f32
-         | (0u << 7)          // A format: E4M3
-         | (0u << 10)         // B format: E4M3
-         | ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-
 // ------------------------------------------------------------------ paired float32 math
 // Two float32 lanes in one 64-bit register (element 0 in the low half); each
 // operation rounds both lanes to nearest even, exactly like its scalar form.
@@ -552,15 +490,6 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
 __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
   return v;
 }
 

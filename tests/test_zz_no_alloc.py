@@ -2,8 +2,9 @@
 
 The allocation-free entry point keeps the K splits' partial down-projections
 in a static device array instead of the caller's workspace; on the same inputs
-it must return the same bytes as the regular call, on two calls in a row (the
-second call reuses the array the first one left behind). This file is
+it must return the same bytes as the regular call, on two calls in a row, each
+right after a call on another activation of the same shape (so every compared
+call finds the array holding someone else's partial sums). This file is
 collected last so it also runs after every other GPU test in one session.
 """
 
@@ -49,8 +50,13 @@ def test_noalloc_matches_the_regular_call_twice(bq, shape):
         L1 = F.bf16_round(rng.normal(0, 0.05, (K, r)))
         L1s = C.bf16_tensor(F.bf16_bits(LO.lowrank_operand(L1, F.rn32(si.cpu().numpy().astype(np.float64)))))
     want = bq.svdq_quantize_act(X, L1s, si, fmt=shape.fmt)
+    # another activation of the same shape: the call before each compared call
+    # leaves its own partial sums in the static array, so a compared call that
+    # skipped writing part of the array would read them and differ
+    X_other = C.bf16_tensor(WL.to_bf16_bits(rng.standard_normal((M, K)) * 3.0))
     assert bq.svdq_check_device_status() == 0
     for call in range(2):
+        bq.svdq_quantize_act_noalloc(X_other, L1s, si, fmt=shape.fmt)
         got = bq.svdq_quantize_act_noalloc(X, L1s, si, fmt=shape.fmt)
         assert bq.svdq_check_device_status() == 0
         for name, a, b in zip(("codes", "scales", "xl1"), got, want):
