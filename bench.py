@@ -45,7 +45,13 @@ import sys
 import threading
 import time
 
-import numpy as np
+# The oracle legs run on every host core this process may use; BLAS thread pools
+# size themselves from the environment when numpy loads, so pin them first.
+HOST_CORES = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+for _var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+    os.environ.setdefault(_var, str(HOST_CORES))
+
+import numpy as np  # noqa: E402
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -57,6 +63,8 @@ UNIT = "TFLOP/s"
 SHAPE = WL.QKV
 AWQ = WL.AWQ_MOD
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, nominal
+AWQ_KERNEL = "awq_gemv_kernel"  # the kernel awq_w4a16_linear runs at the step's 4 tokens
 
 
 def layer_flops(M: int, K: int, N: int, r: int) -> float:
@@ -83,6 +91,116 @@ def quantize_bytes(M: int, K: int, r: int) -> float:
 
 def awq_bytes(M: int, K: int, N: int) -> float:
     return N * K / 2 + N * (K / 64) * 4 + 2.0 * M * K + 2.0 * M * N + 2.0 * N
+
+
+def quantize_bytes_fmt(fmt: str, M: int, K: int, r: int) -> float:
+    """Algorithmic HBM bytes of svdq_quantize_act: X, codes, scales, xl1, L1, smooth_inv."""
+    sc = M * K / 16 if fmt == "nvfp4" else 2.0 * M * K / 64
+    return 2.0 * M * K + M * K / 2 + sc + 4.0 * M * r + 2.0 * K * r + 4.0 * K
+
+
+def median_us(fn, flush, n: int) -> float:
+    """Median device time of fn() in microseconds: n calls, each after the L2
+    flush, with CUDA events on the launch stream right around the call."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n + 3)]
+    for a, b in ev:
+        flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev[3:]) * 1e3
+
+
+def sweep_layers(bq, prep, dev, flush, n: int, fp4_peak: float) -> dict:
+    """The other workloads of the build, each as one SVDQ layer (quantizer, then
+    the 4-bit GEMM with the fused low-rank branch and bias), timed call by call
+    after the flush: the tiny layer, the FLUX-like MLP pair fc1 / fc2 (rank 128,
+    NVFP4) and fc1 in INT4, the rank sweep at hidden 3840 (N 3840 and 15360, rank
+    0 / 32 / 128 / 256; the overhead of the low-rank branch against rank 0), and
+    the QKV projection at batch 4 (M 18432). Weights are prepared on the device
+    from the same seeded draws the tests use; one float32 SVD per weight serves
+    all of its ranks (timing only: parity is pinned on the float64 prep)."""
+    import torch
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    out = {}
+    svd_cache = {}
+    shapes = [WL.TINY, WL.FC1, WL.FC2, WL.FC1_INT4, *WL.RANK_SWEEP, WL.BIG]
+    for sh in shapes:
+        d = WL.svdq_inputs(sh)
+        X = to_dev(d["X"])
+        W = to_dev(d["W"])
+        bias = to_dev(d["bias"]) if d["bias"] is not None else None
+        x_absmax = X.float().abs().amax(dim=0)
+        svd = None
+        if sh.r > 0:
+            key = (sh.seed, sh.N, sh.K)
+            if key not in svd_cache:
+                _, w_hat = prep.smoothed_weight(W, x_absmax)
+                svd_cache[key] = torch.linalg.svd(w_hat.float(), full_matrices=False)
+            svd = svd_cache[key]
+        w = prep.prepare_svdq_weights(W, x_absmax, sh.r, sh.fmt, svd=svd)
+        del W
+        M, K, N, r = sh.M, sh.K, sh.N, sh.r
+        codes = torch.empty(bq.svdq_codes_bytes(sh.fmt, M, K), dtype=torch.uint8, device=dev)
+        scales = torch.empty(bq.svdq_scales_bytes(sh.fmt, M, K), dtype=torch.uint8, device=dev)
+        xl1 = (torch.empty((bq.svdq_xl1_splits(M, K, r), M, r), dtype=torch.float32, device=dev)
+               if r else None)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        quant = lambda: bq.svdq_quantize_act(X, w["L1s"], w["smooth_inv"], fmt=sh.fmt,  # noqa: E731
+                                             codes=codes, scales=scales, xl1=xl1)
+        _, _, xv = quant()
+        gemm = lambda: bq.svdq_w4a4_linear(codes, scales, xv, w["w_codes"], w["w_scales"], w["L2"],  # noqa: E731
+                                           bias, M, N, K, fmt=sh.fmt, Y=Y)
+        t_q = median_us(quant, flush, n)
+        t_g = median_us(gemm, flush, n)
+        f4 = 2.0 * M * N * K
+        e = {"M": M, "K": K, "N": N, "r": r, "format": sh.fmt,
+             "svdq_quantize_act_us": round(t_q, 2),
+             "svdq_quantize_act_gbs": round(quantize_bytes_fmt(sh.fmt, M, K, r) / (t_q * 1e-6) / 1e9, 1),
+             "svdq_w4a4_linear_us": round(t_g, 2),
+             "svdq_w4a4_linear_tflops_4bit": round(f4 / (t_g * 1e-6) / 1e12, 1),
+             "layer_tflops": round(f4 / ((t_q + t_g) * 1e-6) / 1e12, 1)}
+        if sh.fmt == "nvfp4":
+            e["gemm_frac_of_fp4_peak"] = round(f4 / (t_g * 1e-6) / 1e12 / fp4_peak, 3)
+        out[sh.name] = e
+        del X, w, codes, scales, xl1, Y
+        assert bq.svdq_check_device_status() == 0
+    for n_ in (3840, 15360):
+        base = out[f"dit3840_n{n_}_r0"]
+        for r in (32, 128, 256):
+            e = out[f"dit3840_n{n_}_r{r}"]
+            e["lowrank_overhead_gemm"] = round(e["svdq_w4a4_linear_us"] / base["svdq_w4a4_linear_us"] - 1, 3)
+            e["lowrank_overhead_layer"] = round(
+                (e["svdq_w4a4_linear_us"] + e["svdq_quantize_act_us"])
+                / (base["svdq_w4a4_linear_us"] + base["svdq_quantize_act_us"]) - 1, 3)
+    return out
+
+
+def awq_by_tokens(bq, awq_w, bias_a, dev, flush, n: int) -> dict:
+    """The adaLN projection (K 3072, N 18432) at more tokens: the tensor-core
+    GEMM above 64 tokens, and both kernels at 4 and 64 tokens."""
+    import torch
+    out = {}
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    for M in (4, 16, 64, 128, 256):
+        X = torch.randn(M, AWQ.K, device=dev, generator=g).to(torch.bfloat16)
+        Y = torch.empty((M, AWQ.N), dtype=torch.bfloat16, device=dev)
+        for path in ("0", "1"):
+            if path == "0" and M > 64:
+                continue
+            os.environ["SVDQ_AWQ_PATH"] = path
+            t = median_us(lambda: bq.awq_w4a16_linear(X, awq_w["qweight"], awq_w["sz"], bias_a, AWQ.N, Y=Y),
+                          flush, n)
+            name = "gemv" if path == "0" else "tensor_cores"
+            out[f"m{M}_{name}_us"] = round(t, 2)
+            out[f"m{M}_{name}_gbs"] = round(awq_bytes(M, AWQ.K, AWQ.N) / (t * 1e-6) / 1e9, 1)
+        os.environ.pop("SVDQ_AWQ_PATH", None)
+    assert bq.svdq_check_device_status() == 0
+    return out
 
 
 def measured_peaks() -> dict:
@@ -118,6 +236,12 @@ def recorded_traffic(kernel: str) -> float | None:
         if len(parts) >= 3 and parts[0].strip() == kernel and parts[2].strip() == sha:
             return float(parts[1])
     return None
+
+
+def sum_traffic(kernels) -> float | None:
+    """DRAM bytes per call summed over the call's kernels, or None if any is unrecorded."""
+    vals = [recorded_traffic(k) for k in kernels]
+    return None if any(v is None for v in vals) else float(sum(vals))
 
 
 class ClockSampler:
@@ -243,6 +367,34 @@ def time_oracle(host: dict, budget_s: float, rows: int, cols: int,
     return flops, time.perf_counter() - t0, reps
 
 
+def oracle_tiny_layer(budget_s: float) -> dict:
+    """The oracle's whole tiny layer (M 256, K 512, N 512, r 16: a1..a6 with the
+    weights' prep outside the clock), on one BLAS thread and on all of them."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import prep as P
+    from oracle import svdq as S
+    sh = WL.TINY
+    d = WL.svdq_inputs(sh)
+    pr = P.prepare_svdq_layer("nvfp4", d["X"], d["W"], sh.r)
+    flops = layer_flops(sh.M, sh.K, sh.N, sh.r)
+
+    def run():
+        t0, reps = time.perf_counter(), 0
+        while True:
+            S.svdq_forward("nvfp4", d["X"], pr["smooth_inv"], pr["L1"], pr["L2"], pr["w_codes"],
+                           pr["w_scales"], d["bias"])
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                return flops * reps / (time.perf_counter() - t0) / 1e9, reps
+    with threadpool_limits(1):
+        one, reps1 = run()
+    allc, repsn = run()
+    return {"workload": f"{sh.name}: M={sh.M} K={sh.K} N={sh.N} r={sh.r} NVFP4, the whole layer",
+            "gflops_1_thread": round(one, 3), "gflops_all_threads": round(allc, 3),
+            "threads": blas_threads(), "reps": [reps1, repsn]}
+
+
 def awq_plain_host(w_bits: np.ndarray) -> dict:
     from oracle import awq as OA
     from oracle import formats as F
@@ -336,6 +488,8 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle time for the cpu_baseline leg")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the other workloads (for profiling runs of the step)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -494,6 +648,14 @@ def main() -> None:
     t_qkv = sum(e[0].elapsed_time(e[1]) for e in ev3[3:]) / n2
     status = status or bq.svdq_check_device_status()
 
+    # ------------------------------- the other workloads and AWQ at more tokens
+    sweep, awq_tokens = None, None
+    if not args.no_sweep and rank == 0:
+        peaks0 = measured_peaks()
+        sweep = sweep_layers(bq, prep, dev, flush, max(3, min(args.steps, 50)),
+                             peaks0["bf16_tflops"] * FP4_OVER_BF16)
+        awq_tokens = awq_by_tokens(bq, awq_w, bias_a, dev, flush, max(3, min(args.steps, 50)))
+
     # ----------------------------------------------- end to end, host buffers
     Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
     Xh.copy_(X)
@@ -552,7 +714,9 @@ def main() -> None:
                                           "xa_bits": da["X"], "awq_plain": awq_plain_host(da["W"])})
         flops, secs, reps = time_oracle(host, args.cpu_budget, 8, 1152, 1152)
         cpu = {"value": flops / secs / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{reps} x ({sample_text(8, 1152, 1152)}), {secs:.1f} s"}
+               "sample": f"{reps} x ({sample_text(8, 1152, 1152)}), {secs:.1f} s",
+               "host_cores": HOST_CORES,
+               "tiny_layer": oracle_tiny_layer(min(3.0, args.cpu_budget / 4))}
 
     if rank != 0:
         if world > 1:
@@ -577,9 +741,31 @@ def main() -> None:
         "config": config_block(world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp4_peak, "traffic": traffic,
+                     "frac_vs_nominal": achieved / NOMINAL_FP4_TFLOPS,
                      "kernel": "w4a4_nvfp4_gemm_kernel",
-                     "peak_note": f"{peaks['source']} bf16 {peak_kind} x {FP4_OVER_BF16:g} "
-                                  f"(nominal FP4/BF16); vs nominal 9 PFLOP/s: {achieved / 9000:.3f}"},
+                     "peak_note": f"peak = {peaks['source']} bf16 {peak_kind} x {FP4_OVER_BF16:g} "
+                                  f"(nominal FP4/BF16 ratio; no FP4 peak is measured), so frac is of the "
+                                  f"measured-bf16-scaled FP4 peak; frac_vs_nominal is of the nominal dense "
+                                  f"FP4 {NOMINAL_FP4_TFLOPS:g} TFLOP/s"},
+        "roofline_hbm": {
+            "svdq_quantize_act": {
+                "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                "achieved": quantize_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9,
+                "frac": quantize_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "algorithmic_bytes": quantize_bytes(M, K, r),
+                "traffic": sum_traffic(("quantize_act_kernel", "xl1_reduce_kernel")),
+                "kernels": "quantize_act_kernel + xl1_reduce_kernel (K-split partial sums)",
+                "us": k1_ms * 1e3},
+            "awq_w4a16_linear": {
+                "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                "achieved": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / (k3_ms * 1e-3) / 1e9,
+                "frac": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / (k3_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "algorithmic_bytes": awq_bytes(AWQ.M, AWQ.K, AWQ.N),
+                "traffic": sum_traffic((AWQ_KERNEL,)),
+                "kernels": AWQ_KERNEL,
+                "us": k3_ms * 1e3},
+            "peak_note": f"{peaks['source']} HBM copy bandwidth; achieved = algorithmic bytes / "
+                         f"event-to-event time in the kernel-timing pass"},
         "cpu_baseline": cpu,
         "e2e": {"value": job_tflops(step_flops(), world, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2 + Xa.numel() * 2,
@@ -615,6 +801,15 @@ def main() -> None:
         },
         "device_status": status,
     }
+    if sweep is not None:
+        out["kernels"]["workloads"] = {
+            "timing": "each layer's quantizer and GEMM called alone after the L2 flush, event to event, "
+                      "median of the calls",
+            **sweep}
+        out["kernels"]["awq_by_tokens"] = {
+            "timing": f"awq_w4a16_linear at K={AWQ.K} N={AWQ.N}, event to event after the flush, median; "
+                      f"the GEMV (warp-level MMA) serves M <= 64, the tensor-core GEMM any M",
+            **awq_tokens}
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()

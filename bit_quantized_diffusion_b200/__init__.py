@@ -184,6 +184,53 @@ def svdq_w4a4_linear(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, M: int
     return Y
 
 
+def svdq_mlp_splits(M: int, N1: int) -> int:
+    """S: svdq_mlp_fc1's xl1_2 buffer holds S x M x r2 float32 (its working space)."""
+    return N.load().svdq_mlp_splits(M, N1)
+
+
+def svdq_mlp_fc1(a_codes, a_scales, xl1_1, w_codes, w_scales, L2_1, bias1, smooth_inv2, L1t_2,
+                 M: int, N1: int, K1: int, codes2=None, scales2=None, xl1_2=None, hhat=None, stream=None):
+    """The fused MLP's fc1 (NVFP4): fc1's layer, GELU (tanh form), fc2's smoothing and
+    fc2's activation quantization and down-projection in the epilogue. L1t_2 is fc2's
+    factor transposed, bf16 [r2, N1] (or None for r2 = 0). hhat, if given, receives
+    h_hat float32 [M, N1]. Returns (codes2, scales2, xl1_2 [M, r2] or None): fc2's input."""
+    lib = N.load()
+    r1 = 0 if L2_1 is None else L2_1.shape[0]
+    r2 = 0 if L1t_2 is None else L1t_2.shape[0]
+    dev = a_codes.device
+    if r1 and (xl1_1 is None or xl1_1.dtype != torch.float32 or xl1_1.numel() < M * r1):
+        raise ValueError("xl1_1 must be float32 [M, r1]")
+    if r1 and (L2_1.dtype != torch.bfloat16 or tuple(L2_1.shape) != (r1, N1)):
+        raise ValueError("L2_1 must be bf16 [r1, N1]")
+    if r2 and (L1t_2.dtype != torch.bfloat16 or tuple(L1t_2.shape) != (r2, N1)):
+        raise ValueError("L1t_2 must be bf16 [r2, N1]")
+    if smooth_inv2 is not None and (smooth_inv2.dtype != torch.float32 or smooth_inv2.numel() != N1):
+        raise ValueError("smooth_inv2 must be float32 [N1]")
+    if bias1 is not None and (bias1.dtype != torch.bfloat16 or bias1.numel() != N1):
+        raise ValueError("bias1 must be bf16 [N1]")
+    S = lib.svdq_mlp_splits(M, N1)
+    if S < 1:
+        raise ValueError("N1 must be a positive multiple of 128")
+    if codes2 is None:
+        codes2 = torch.empty(lib.svdq_codes_bytes(N.NVFP4_G16, M, N1), dtype=torch.uint8, device=dev)
+    if scales2 is None:
+        scales2 = torch.empty(lib.svdq_scales_bytes(N.NVFP4_G16, M, N1), dtype=torch.uint8, device=dev)
+    _need(codes2, lib.svdq_codes_bytes(N.NVFP4_G16, M, N1), "codes2")
+    _need(scales2, lib.svdq_scales_bytes(N.NVFP4_G16, M, N1), "scales2")
+    if r2 and xl1_2 is None:
+        xl1_2 = torch.empty((S, M, r2), dtype=torch.float32, device=dev)
+    if r2 and (xl1_2.dtype != torch.float32 or xl1_2.numel() < S * M * r2):
+        raise ValueError(f"xl1_2 must be float32 [{S}, M, r2]")
+    if hhat is not None and (hhat.dtype != torch.float32 or hhat.numel() < M * N1):
+        raise ValueError("hhat must be float32 [M, N1]")
+    N.check(lib.svdq_mlp_fc1(M, N1, K1, r1, r2, _ptr(a_codes), _ptr(a_scales), _ptr(xl1_1) if r1 else None,
+                             _ptr(w_codes), _ptr(w_scales), _ptr(L2_1), _ptr(bias1), _ptr(smooth_inv2),
+                             _ptr(L1t_2), _ptr(codes2), _ptr(scales2), _ptr(xl1_2) if r2 else None,
+                             _ptr(hhat), _stream(stream)), "svdq_mlp_fc1")
+    return codes2, scales2, (xl1_2.view(-1)[:M * r2].view(M, r2) if r2 else None)
+
+
 def svdq_w4a4_linear_qkv_norm_rope(a_codes, a_scales, xl1, w_codes, w_scales, L2, bias, norm_q,
                                    norm_k, rope_cos, rope_sin, M: int, N_: int, K: int,
                                    eps: float = 1e-6, out_dtype=torch.bfloat16,
@@ -331,6 +378,85 @@ def awq_w4a16_linear(X: torch.Tensor, qweight: torch.Tensor, sz: torch.Tensor,
     N.check(lib.awq_w4a16_linear(M, N_, K, group, _ptr(X), _ptr(qweight), _ptr(sz), _ptr(bias),
                                  _ptr(Y), _stream(stream)), "awq_w4a16_linear")
     return Y
+
+
+def svdq_column_absmax(A: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """absmax [K] float32 = max over rows of |A| for a 2-D bf16 tensor A [rows, K]."""
+    lib = N.load()
+    if A.dtype != torch.bfloat16 or A.dim() != 2:
+        raise ValueError("A must be a 2-D bf16 tensor")
+    rows, K = A.shape
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=A.device)
+    if out.dtype != torch.float32 or out.numel() != K:
+        raise ValueError("out must be float32 [K]")
+    N.check(lib.svdq_column_absmax(rows, K, _ptr(A), K, _ptr(out), _stream(stream)), "svdq_column_absmax")
+    return out
+
+
+def svdq_smoothing(x_absmax: torch.Tensor, W: torch.Tensor, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """smooth_inv [K] float32 = RN32(1 / lambda), lambda = sqrt(x_absmax / max_n |W[n]|)
+    in float64 (1 where either maximum is 0)."""
+    lib = N.load()
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 tensor")
+    Nr, K = W.shape
+    if x_absmax.dtype != torch.float32 or x_absmax.numel() != K:
+        raise ValueError("x_absmax must be float32 [K]")
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=W.device)
+    N.check(lib.svdq_smoothing(Nr, K, _ptr(x_absmax), _ptr(W), _ptr(out), _stream(stream)), "svdq_smoothing")
+    return out
+
+
+def svdq_lowrank_factors(U: torch.Tensor, S: torch.Tensor, Vh: torch.Tensor, r: int, stream=None):
+    """(L1 [K, r], L2 [r, N]) bf16 from the float64 SVD W_hat = U diag(S) Vh, each element
+    rounded once: L1 = RN_bf16(Vh[:r]^T sqrt(S_r)), L2 = RN_bf16(sqrt(S_r) U[:, :r]^T)."""
+    lib = N.load()
+    if U.dtype != torch.float64 or S.dtype != torch.float64 or Vh.dtype != torch.float64:
+        raise ValueError("U, S, Vh must be float64")
+    U, S, Vh = U.contiguous(), S.contiguous(), Vh.contiguous()
+    Nr, K = U.shape[0], Vh.shape[1]
+    L1 = torch.empty((K, r), dtype=torch.bfloat16, device=U.device)
+    L2 = torch.empty((r, Nr), dtype=torch.bfloat16, device=U.device)
+    N.check(lib.svdq_lowrank_factors(Nr, K, r, _ptr(U), U.shape[1], _ptr(S), _ptr(Vh), K, _ptr(L1),
+                                     _ptr(L2), _stream(stream)), "svdq_lowrank_factors")
+    return L1, L2
+
+
+def svdq_residual(W: torch.Tensor, smooth_inv: torch.Tensor, L1: torch.Tensor | None,
+                  L2: torch.Tensor | None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """R [N, K] bf16 = RN_bf16(W diag(1 / smooth_inv) - (L1 L2)^T), float64 inside."""
+    lib = N.load()
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 tensor")
+    Nr, K = W.shape
+    r = 0 if L1 is None else L1.shape[1]
+    if r and (L1.dtype != torch.bfloat16 or tuple(L1.shape) != (K, r) or L2 is None
+              or L2.dtype != torch.bfloat16 or tuple(L2.shape) != (r, Nr)):
+        raise ValueError("L1 must be bf16 [K, r] and L2 bf16 [r, N]")
+    if smooth_inv.dtype != torch.float32 or smooth_inv.numel() != K:
+        raise ValueError("smooth_inv must be float32 [K]")
+    if out is None:
+        out = torch.empty((Nr, K), dtype=torch.bfloat16, device=W.device)
+    N.check(lib.svdq_residual(Nr, K, r, _ptr(W), _ptr(smooth_inv), _ptr(L1), _ptr(L2) if r else None,
+                              _ptr(out), _stream(stream)), "svdq_residual")
+    return out
+
+
+def awq_quantize_weight(W: torch.Tensor, stream=None):
+    """The AWQ int4 g64 quantizer of W [N, K] bf16, straight into the tiled layouts
+    awq_w4a16_linear reads. Returns (qweight, sz) as uint8 tensors."""
+    lib = N.load()
+    if W.dtype != torch.bfloat16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D bf16 tensor")
+    Nr, K = W.shape
+    qt = torch.empty(lib.awq_qweight_bytes(Nr, K), dtype=torch.uint8, device=W.device)
+    szt = torch.empty(lib.awq_sz_bytes(Nr, K), dtype=torch.uint8, device=W.device)
+    N.check(lib.awq_quantize_weight(Nr, K, _ptr(W), _ptr(qt), _ptr(szt), _stream(stream)),
+            "awq_quantize_weight")
+    return qt, szt
 
 
 def svdq_pack(kind, fmt, rows: int, K: int, plain_codes, plain_scales, plain_zeros=None,

@@ -26,6 +26,8 @@ EXPORTS = (
     "svdq_debug_wait_timeout", "svdq_pack_lowrank", "svdq_xl1_splits",
     "svdq_quantize_act_noalloc", "svdq_tensor_scale", "svdq_quantize_act_two_level",
     "svdq_w4a4_linear_two_level", "svdq_w4a4_linear_qkv_norm_rope",
+    "svdq_column_absmax", "svdq_smoothing", "svdq_lowrank_factors", "svdq_residual",
+    "awq_quantize_weight", "svdq_mlp_splits", "svdq_mlp_fc1",
 )
 
 _lib = None
@@ -67,6 +69,13 @@ def load() -> ctypes.CDLL:
                                             _P, _I, _I, _P]),
         "svdq_w4a4_linear_qkv_norm_rope": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                 ctypes.c_float, _P, _P, _P, _I, _I, _P]),
+        "svdq_column_absmax": (_I, [_I, _I, _P, _I, _P, _P]),
+        "svdq_smoothing": (_I, [_I, _I, _P, _P, _P, _P]),
+        "svdq_lowrank_factors": (_I, [_I, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P]),
+        "svdq_residual": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _P]),
+        "awq_quantize_weight": (_I, [_I, _I, _P, _P, _P, _P]),
+        "svdq_mlp_splits": (_I, [_I, _I]),
+        "svdq_mlp_fc1": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

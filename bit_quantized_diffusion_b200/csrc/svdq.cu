@@ -13,8 +13,11 @@
 
 #include "../../include/svdq.h"
 #include "awq.cuh"
+#include "awq_gemm.cuh"
 #include "int4_gemm.cuh"
+#include "mlp_fc1.cuh"
 #include "pack.cuh"
+#include "prep.cuh"
 #include "quantize_act.cuh"
 #include "w4a4_gemm.cuh"
 
@@ -38,6 +41,7 @@ struct DeviceInfo {
   int num_sms = 0;
   int gemm_pairs = 0;  // co-resident clusters of the CTA-pair NVFP4 GEMM
   int int4_pairs = 0;  // the same for the INT4 GEMM
+  int mlp_pairs = 0;   // the same for the fused MLP's fc1
   int gemm_pair_mode = -1;  // -1: by shape; SVDQ_GEMM_PAIR=0/1 forces single-CTA / CTA-pair tiles
   uint32_t* status = nullptr;
   float* xl1_scratch = nullptr;  // device address of g_xl1_scratch
@@ -129,7 +133,9 @@ svdq_status device_setup(DeviceInfo** out) {
     if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_int4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kI4SmemBytes)) != cudaSuccess)
+                             static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_mlp_fc1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kMlSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     // all of the SM's unified L1/shared storage as shared memory, so that the
     // occupancy the host code plans for (e.g. two quantizer CTAs per SM) is real
@@ -141,12 +147,16 @@ svdq_status device_setup(DeviceInfo** out) {
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true, true>),
                           reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<false>),
                           reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<true>),
+                          reinterpret_cast<const void*>(awq_gemm_kernel),
+                          reinterpret_cast<const void*>(w4a4_mlp_fc1_kernel),
                           reinterpret_cast<const void*>(awq_gemv_kernel<1>),
                           reinterpret_cast<const void*>(awq_gemv_kernel<2>)})
       if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return SVDQ_ERR_CUDA;
-    if (cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(awq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(awq_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess ||
         cudaFuncSetAttribute(awq_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess)
@@ -175,6 +185,7 @@ svdq_status device_setup(DeviceInfo** out) {
       };
       d.gemm_pairs = pairs(w4a4_nvfp4_gemm_kernel<true>, kGmThreads, GmCfg<true>::kSmemBytes);
       d.int4_pairs = pairs(w4a4_int4_gemm_kernel<true>, kI4Threads, kI4SmemBytes);
+      d.mlp_pairs = pairs(w4a4_mlp_fc1_kernel, kMlThreads, kMlSmemBytes);
       if (std::getenv("SVDQ_DEBUG") != nullptr)
         std::fprintf(stderr, "svdq: %d SMs, %d / %d co-resident NVFP4 / INT4 GEMM CTA pairs\n",
                      d.num_sms, d.gemm_pairs, d.int4_pairs);
@@ -300,6 +311,49 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
            : launch_kernel(d, w4a4_int4_gemm_kernel<false>, dim3(units), dim3(kI4Threads),
                            kI4SmemBytes, stream, 1, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p);
   if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// AWQ W4A16 on the tensor cores (awq_gemm_kernel): token tiles of T = M rounded
+// up to 16 (at most 128), 128 weight rows per tile, one persistent CTA per SM;
+// weights and (s, z) in the fragment order of svdq_pack(AWQ).
+svdq_status launch_awq_gemm(const DeviceInfo* d, int M, int N, int K, const void* X,
+                            const void* qweight, const void* sz, const void* bias, void* Y,
+                            cudaStream_t stream) {
+  const int T = M >= kAgMaxT ? kAgMaxT : (M + 15) / 16 * 16;
+  const int tb = T <= 32 ? 32 : (T <= 64 ? 64 : 128);
+  int stages = kAgMaxStages;
+  while (stages > 2 && ag_smem_bytes(T, stages) > 232448) --stages;
+  const int G = K / 64, nblocks = (N + 15) / 16;
+  CUtensorMap tm_q, tm_sz, tm_x;
+  if (!make_tmap_3d_u64(&tm_q, qweight, 64, G, nblocks, 1, 8) ||
+      !make_tmap_3d_u64(&tm_sz, sz, 8, G, nblocks, 1, 8) ||
+      !make_tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64,
+                    T, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  AgParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.T = T;
+  p.tb = tb;
+  p.nbuf = 512 / tb;
+  p.stages = stages;
+  p.tiles_m = (M + kAgMaxT - 1) / kAgMaxT;
+  p.tiles = p.tiles_m * ((N + kAgRows - 1) / kAgRows);
+  p.sz = static_cast<const uint32_t*>(sz);
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.status = d->status;
+  const int grid = p.tiles < d->num_sms ? p.tiles : d->num_sms;
+  if (debug_on())
+    std::fprintf(stderr, "awq_w4a16_linear (tensor cores): M=%d N=%d K=%d T=%d stages=%d tiles=%d grid=%d\n",
+                 M, N, K, T, stages, p.tiles, grid);
+  if (launch_kernel(d, awq_gemm_kernel, dim3(grid), dim3(kAgThreads), ag_smem_bytes(T, stages), stream, 1,
+                    tm_q, tm_sz, tm_x, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }
@@ -623,6 +677,106 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(int M, int N, int K, int r, const voi
                           L2, bias, Y, ldy, out, stream, nullptr, nullptr, &qk);
 }
 
+int svdq_mlp_splits(int M, int N1) {
+  if (M < 1 || N1 < kMlBN || N1 % kMlBN) return 0;
+  DeviceInfo* d = nullptr;
+  if (device_setup(&d) != SVDQ_OK) return 0;
+  const int row_blocks = (M + 2 * kMlBM - 1) / (2 * kMlBM), ntn = N1 / kMlBN;
+  int nsplit = d->mlp_pairs / row_blocks;
+  if (nsplit < 1) nsplit = 1;
+  if (nsplit > 8) nsplit = 8;
+  if (nsplit > ntn) nsplit = ntn;
+  const int tps = (ntn + nsplit - 1) / nsplit;
+  return (ntn + tps - 1) / tps;
+}
+
+svdq_status svdq_mlp_fc1(int M, int N1, int K1, int r1, int r2, const void* a_codes, const void* a_scales,
+                         const float* xl1_1, const void* w_codes, const void* w_scales, const void* L2_1,
+                         const void* bias1, const float* smooth_inv2, const void* L1t_2, void* codes2,
+                         void* scales2, float* xl1_2, float* hhat, svdq_stream_t stream) {
+  if (M < 1 || N1 < kMlBN || N1 % kMlBN || K1 < 64 || K1 % 64 || !rank_ok(r1)) return SVDQ_ERR_INVALID_ARG;
+  if (r2 < 0 || r2 > kMlR2Max || r2 % 32) return SVDQ_ERR_INVALID_ARG;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !codes2 || !scales2) return SVDQ_ERR_INVALID_ARG;
+  if ((r1 > 0) != (xl1_1 != nullptr) || (r1 > 0) != (L2_1 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if ((r2 > 0) != (L1t_2 != nullptr) || (r2 > 0) != (xl1_2 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(codes2) || !aligned16(scales2) || (xl1_1 && !aligned16(xl1_1)) || (L2_1 && !aligned16(L2_1)) ||
+      (L1t_2 && !aligned16(L1t_2)) || (xl1_2 && !aligned16(xl1_2)) || (hhat && !aligned16(hhat)) ||
+      (smooth_inv2 && (reinterpret_cast<uintptr_t>(smooth_inv2) & 3u)) ||
+      (bias1 && (reinterpret_cast<uintptr_t>(bias1) & 1u)))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const uint64_t kb = static_cast<uint64_t>(K1 / 64);
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_l2, tm_xl1, tm_l1t;
+  if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K1 / 2, M, K1 / 2, 128, kMlBM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K1 / 2, N1, K1 / 2, 128, kMlBRows,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_scales, 256, pad128(M) / 128 * kb * 2, 256, 256,
+                    8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tm_sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 256, pad128(N1) / 128 * kb * 2, 256,
+                    256, 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ERR_CUDA;
+  if (r1 > 0) {
+    if (!make_tmap_2d(&tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2_1, N1, r1, static_cast<uint64_t>(N1) * 2,
+                      64, kMlLrK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xl1_1, r1, M, static_cast<uint64_t>(r1) * 4,
+                      kMlLrK, kMlBM, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l2 = tm_a;
+    tm_xl1 = tm_a;
+  }
+  if (r2 > 0) {
+    // L1_2^T [r2, N1] bf16: 64-column boxes of this CTA's r2 / 2 ranks
+    if (!make_tmap_2d(&tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t_2, N1, r2, static_cast<uint64_t>(N1) * 2,
+                      64, r2 / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tm_l1t = tm_a;
+  }
+  MlpParams p;
+  p.M = M;
+  p.N1 = N1;
+  p.K1 = K1;
+  p.r1 = r1;
+  p.r2 = r2;
+  p.row_blocks = (M + 2 * kMlBM - 1) / (2 * kMlBM);
+  p.ntn = N1 / kMlBN;
+  p.nsplit = svdq_mlp_splits(M, N1);
+  p.tps = (p.ntn + p.nsplit - 1) / p.nsplit;
+  p.units = p.row_blocks * p.nsplit;
+  p.bias1 = static_cast<const __nv_bfloat16*>(bias1);
+  p.smooth_inv2 = smooth_inv2;
+  p.codes2 = static_cast<uint8_t*>(codes2);
+  p.scales2 = static_cast<uint8_t*>(scales2);
+  p.xl1_part = xl1_2;
+  p.hhat = hhat;
+  p.status = d->status;
+  const int pairs = p.units < d->mlp_pairs ? p.units : d->mlp_pairs;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (debug_on())
+    std::fprintf(stderr, "svdq_mlp_fc1: M=%d N1=%d K1=%d r1=%d r2=%d units=%d (splits %d, %d tiles each) pairs=%d\n",
+                 M, N1, K1, r1, r2, p.units, p.nsplit, p.tps, pairs);
+  if (launch_kernel(d, w4a4_mlp_fc1_kernel, dim3(2 * pairs), dim3(kMlThreads), kMlSmemBytes, cs, 2, tm_a, tm_b,
+                    tm_sfa, tm_sfb, tm_l2, tm_xl1, tm_l1t, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  if (r2 > 0 && p.nsplit > 1) {
+    // xl1_2[0] += xl1_2[1] + ... in order
+    const size_t n4 = static_cast<size_t>(M) * r2 / 4;
+    if (launch_kernel(d, xl1_reduce_kernel, dim3(grid_for(n4, 256)), dim3(256), 0, cs, 1,
+                      reinterpret_cast<float4*>(xl1_2), reinterpret_cast<const float4*>(xl1_2 + static_cast<size_t>(M) * r2),
+                      p.nsplit, n4) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+  }
+  return launch_status();
+}
+
 svdq_status svdq_tensor_scale(int M, int K, const void* X, int ldx, const float* smooth_inv,
                               float* scale, svdq_stream_t stream) {
   if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8 || !X || !scale) return SVDQ_ERR_INVALID_ARG;
@@ -661,14 +815,18 @@ svdq_status svdq_quantize_act_two_level(int M, int K, int r, const void* X, int 
 
 svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, const void* qweight,
                              const void* sz, const void* bias, void* Y, svdq_stream_t stream) {
-  if (group != 64 || M < 1 || M > kAwqMaxM || N < 1 || K < 64 || K % 64)
-    return SVDQ_ERR_INVALID_ARG;
+  if (group != 64 || M < 1 || N < 1 || K < 64 || K % 64) return SVDQ_ERR_INVALID_ARG;
   if (!X || !qweight || !sz || !Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(qweight) || !aligned16(sz) || !aligned16(Y) ||
       (bias && (reinterpret_cast<uintptr_t>(bias) & 1)))
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
   if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  // the path by M; SVDQ_AWQ_PATH=0 / 1 forces the GEMV / the tensor-core GEMM (read per call)
+  const char* force = std::getenv("SVDQ_AWQ_PATH");
+  const bool gemm = force != nullptr ? std::atoi(force) != 0 : M > kAwqMaxM;
+  if (gemm) return launch_awq_gemm(d, M, N, K, X, qweight, sz, bias, Y, static_cast<cudaStream_t>(stream));
+  if (M > kAwqMaxM) return SVDQ_ERR_UNSUPPORTED;  // the GEMV was forced
   // tokens per launch: at most 16 (two 8-token MMA blocks), and as many X rows
   // as fit in shared memory beside a weight ring of at least two stages
   const size_t smem_cap = 232448;
@@ -838,6 +996,83 @@ svdq_status svdq_pack_lowrank(int K, int r, const void* L1, const float* smooth_
   const size_t n = static_cast<size_t>(K) * r;
   pack_lowrank_kernel<<<grid_for(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(L1), smooth_inv, static_cast<__nv_bfloat16*>(L1s), K, r);
+  return launch_status();
+}
+
+svdq_status svdq_column_absmax(int rows, int K, const void* A, int lda, float* absmax,
+                               svdq_stream_t stream) {
+  if (rows < 1 || K < 8 || K % 8 || lda < K || lda % 8 || !A || !absmax) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(A) || (reinterpret_cast<uintptr_t>(absmax) & 3u)) return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(absmax, 0, static_cast<size_t>(K) * sizeof(float), cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  // at least one thread per 8 columns; the rows are split among the rest
+  const size_t units = static_cast<size_t>(K / 8);
+  unsigned grid = grid_for(units * static_cast<size_t>(rows), 256);
+  if (grid > static_cast<unsigned>(4 * d->num_sms)) grid = 4 * d->num_sms;
+  const unsigned min_grid = static_cast<unsigned>((units + 255) / 256);
+  if (grid < min_grid) grid = min_grid;
+  column_absmax_kernel<<<grid, 256, 0, cs>>>(static_cast<const uint16_t*>(A), rows, K, lda,
+                                             reinterpret_cast<uint32_t*>(absmax));
+  return launch_status();
+}
+
+svdq_status svdq_smoothing(int N, int K, const float* x_absmax, const void* W, float* smooth_inv,
+                           svdq_stream_t stream) {
+  if (N < 1 || K < 8 || K % 8 || !x_absmax || !W || !smooth_inv) return SVDQ_ERR_INVALID_ARG;
+  if (svdq_status st = svdq_column_absmax(N, K, W, K, smooth_inv, stream); st != SVDQ_OK) return st;
+  smoothing_kernel<<<(K + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x_absmax, smooth_inv, K);
+  return launch_status();
+}
+
+svdq_status svdq_lowrank_factors(int N, int K, int r, const double* U, int ldu, const double* S,
+                                 const double* Vh, int ldvh, void* L1, void* L2, svdq_stream_t stream) {
+  if (N < 1 || K < 1 || r < 1 || r > N || r > K || ldu < r || ldvh < K) return SVDQ_ERR_INVALID_ARG;
+  if (!U || !S || !Vh || !L1 || !L2) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(U) & 7u) || (reinterpret_cast<uintptr_t>(S) & 7u) ||
+      (reinterpret_cast<uintptr_t>(Vh) & 7u) || (reinterpret_cast<uintptr_t>(L1) & 1u) ||
+      (reinterpret_cast<uintptr_t>(L2) & 1u))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const size_t total = static_cast<size_t>(K) * r + static_cast<size_t>(r) * N;
+  lowrank_factors_kernel<<<grid_for(total, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      U, ldu, S, Vh, ldvh, static_cast<uint16_t*>(L1), static_cast<uint16_t*>(L2), N, K, r);
+  return launch_status();
+}
+
+svdq_status svdq_residual(int N, int K, int r, const void* W, const float* smooth_inv, const void* L1,
+                          const void* L2, void* R, svdq_stream_t stream) {
+  if (N < 1 || K < 1 || r < 0 || r > 4096 || !W || !smooth_inv || !R) return SVDQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1 != nullptr) || (r > 0) != (L2 != nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(W) & 1u) || (reinterpret_cast<uintptr_t>(R) & 1u) ||
+      (reinterpret_cast<uintptr_t>(smooth_inv) & 3u) || (reinterpret_cast<uintptr_t>(L1) & 1u) ||
+      (reinterpret_cast<uintptr_t>(L2) & 1u))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const dim3 grid((K + kResTile - 1) / kResTile, (N + kResTile - 1) / kResTile);
+  residual_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), smooth_inv, static_cast<const uint16_t*>(L1),
+      static_cast<const uint16_t*>(L2), static_cast<uint16_t*>(R), N, K, r);
+  return launch_status();
+}
+
+svdq_status awq_quantize_weight(int N, int K, const void* W, void* qweight, void* sz,
+                                svdq_stream_t stream) {
+  if (N < 1 || K < 64 || K % 64 || !W || !qweight || !sz) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(W) & 1u) || !aligned16(qweight) || !aligned16(sz))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (svdq_status st = device_setup(&d); st != SVDQ_OK) return st;
+  const size_t blocks = static_cast<size_t>((N + 15) / 16) * (K / 64);
+  if (blocks > 0x7FFFFFFFull) return SVDQ_ERR_UNSUPPORTED;
+  awq_quantize_kernel<<<static_cast<unsigned>(blocks), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), N, K, static_cast<uint32_t*>(qweight), static_cast<uint32_t*>(sz));
   return launch_status();
 }
 

@@ -16,9 +16,11 @@
  * up-projection (svdq_w4a4_linear), NVFP4 with a per-tensor second scale level
  * (svdq_tensor_scale, svdq_quantize_act_two_level, svdq_w4a4_linear_two_level),
  * the fused QKV projection with head norm and rotation
- * (svdq_w4a4_linear_qkv_norm_rope), the AWQ W4A16 linear (awq_w4a16_linear),
- * layout conversion (svdq_pack, svdq_unpack, svdq_pack_lowrank), buffer sizes,
- * and the device status word (svdq_check_device_status).
+ * (svdq_w4a4_linear_qkv_norm_rope), the fused MLP's fc1 (svdq_mlp_fc1), the AWQ W4A16 linear (awq_w4a16_linear),
+ * layout conversion (svdq_pack, svdq_unpack, svdq_pack_lowrank), offline weight
+ * preparation (svdq_column_absmax, svdq_smoothing, svdq_lowrank_factors,
+ * svdq_residual, awq_quantize_weight), buffer sizes, and the device status word
+ * (svdq_check_device_status).
  *
  * Conventions for every call:
  *  - Memory: the caller allocates and owns every buffer. Pointers named as device
@@ -30,7 +32,8 @@
  *  - Errors: argument errors are detected on the host before any launch and
  *    returned synchronously; nothing is launched then. A failed launch returns
  *    SVDQ_ERR_CUDA. A kernel whose bounded wait ran out records it in a device
- *    status word, read (and cleared) by svdq_check_device_status.
+ *    status word, read (and cleared) by svdq_check_device_status; the outputs
+ *    of every call enqueued since the previous check are then undefined.
  *  - Matrices are row-major. bf16/fp16 are IEEE-style 16-bit patterns.
  *  - Shapes: M >= 1; K % 64 == 0; N % 16 == 0; r == 0 or (r % 16 == 0 and r <= 256).
  */
@@ -143,16 +146,25 @@ svdq_status svdq_quantize_act(svdq_format format, int M, int K, int r, const voi
  * down-projections of K splits 1 .. S-1 go to a working array the library
  * holds in device memory for each device (one static array of 2^21 float32,
  * 8 MiB; nothing is allocated or freed at any time). The pages describe no
- * counterpart of this call: it exists for callers that must not hand the
- * library any memory beyond the inputs and outputs.
+ * counterpart of this call. It exists for callers that cannot allocate device
+ * memory at the point where they quantize: a serving runtime or a plugin of a
+ * host framework whose allocator owns all device memory and sizes it before the
+ * first request, so that a cudaMalloc mid-step would go around that budget, may
+ * block or synchronise the device, and may fail under memory pressure. Such a
+ * caller passes only the inputs and outputs it already holds.
+ *
+ * Set-up: the first call of any entry point of this library on a device (this
+ * one included) looks up that device's copy of the array (cudaGetSymbolAddress
+ * with the device current) and sets kernel attributes, once per device; make
+ * that first call before any stream capture begins on the device.
  *
  * Limit: (S - 1) * M * r <= 2^21 with S = svdq_xl1_splits(M, K, r); a larger
  * request returns SVDQ_ERR_UNSUPPORTED before anything is launched (r == 0 always
  * fits). Nothing in the array needs to start at zero: each call writes every
- * element it reads. The array is shared by all calls on a device, so two of
- * these calls in flight at the same time (e.g. on different streams) race;
- * calls ordered on one stream do not. Other arguments, layouts and errors as
- * for svdq_quantize_act.
+ * element it reads. The array is shared by all calls on a device and keeps
+ * the last call's partial sums, so two of these calls that overlap on the GPU
+ * (e.g. in flight on different streams) race on it; calls ordered on one
+ * stream do not. Other arguments, layouts and errors as for svdq_quantize_act.
  */
 svdq_status svdq_quantize_act_noalloc(svdq_format format, int M, int K, int r, const void* X,
                                       int ldx, const float* smooth_inv, const void* L1s,
@@ -236,6 +248,44 @@ svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a
                                        void* Y, int ldy, svdq_out out, svdq_stream_t stream);
 
 /*
+ * svdq_mlp_fc1 -- the first half of the fused MLP (Diffusers blog, "From SVDQuant
+ * to Nunchaku Lite": the original engine runs GELU/MLP as one fused path, where
+ * Lite runs the two SVDQ linears apart). fc1's NVFP4 layer, and in its epilogue
+ * everything fc2 needs from the hidden activation, so the [M, N1] activation never
+ * reaches HBM in 16 bits:
+ *
+ *   y1     = the fc1 layer as svdq_w4a4_linear computes it, float32 in tensor memory
+ *   h_hat  = RN32(RN32(GELU(RN32(y1))) * smooth_inv2[n]),
+ *            GELU(y) = 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) in float32
+ *   codes2, scales2 = NVFP4 codes and scales of h_hat (steps a2, a3 of fc2, groups of 16
+ *            along N1, the layouts svdq_quantize_act writes)
+ *   xl1_2  = h_hat L1_2 (step a4 of fc2; h_hat as a bf16 hi + lo pair on the tensor
+ *            cores, float32 accumulation)
+ *
+ * Then svdq_w4a4_linear(NVFP4, M, N2, K = N1, r2, codes2, scales2, xl1_2, ...) is fc2.
+ *
+ * a_codes, a_scales, xl1_1  fc1's input from svdq_quantize_act (M rows, K1)
+ * w_codes, w_scales         fc1's weight codes/scales (N1 rows)
+ * L2_1                      device, bf16 [r1, N1]; NULL iff r1 == 0
+ * bias1                     device, bf16 [N1] or NULL
+ * smooth_inv2               device, float32 [N1] (fc2's smoothing) or NULL (1)
+ * L1t_2                     device, bf16 [r2, N1]: fc2's factor L1_2 [N1, r2] transposed
+ *                           (row j holds column j of L1_2); NULL iff r2 == 0
+ * codes2, scales2           device, svdq_codes_bytes / svdq_scales_bytes(NVFP4, M, N1), written
+ * xl1_2                     device, float32, svdq_mlp_splits(M, N1) * M * r2 elements of
+ *                           working space; on return its first M * r2 hold xl1_2 [M, r2].
+ *                           NULL iff r2 == 0
+ * hhat                      device, float32 [M, N1] receiving h_hat, or NULL (for tests)
+ * Shapes: N1 % 128 == 0, K1 % 64 == 0, r1 as for svdq_w4a4_linear, r2 in {0, 32, 64, 96, 128}.
+ * INVALID_ARG / ALIGNMENT before any launch otherwise.
+ */
+int svdq_mlp_splits(int M, int N1);
+svdq_status svdq_mlp_fc1(int M, int N1, int K1, int r1, int r2, const void* a_codes, const void* a_scales,
+                         const float* xl1_1, const void* w_codes, const void* w_scales, const void* L2_1,
+                         const void* bias1, const float* smooth_inv2, const void* L1t_2, void* codes2,
+                         void* scales2, float* xl1_2, float* hhat, svdq_stream_t stream);
+
+/*
  * svdq_w4a4_linear_qkv_norm_rope -- the fused QKV projection of an attention
  * block with its head normalisation and rotary embedding in the GEMM's epilogue
  * (Diffusers blog, the fused QKV section: to_q, to_k, to_v joined along the
@@ -266,20 +316,27 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(int M, int N, int K, int r, const voi
                                            void* Y, int ldy, svdq_out out, svdq_stream_t stream);
 
 /*
- * awq_w4a16_linear -- step a7, the AWQ W4A16 linear for small-M modulation
- * projections (Diffusers blog, "From SVDQuant to Nunchaku Lite": awq_w4a16 for
- * the memory-bound adaptive-norm projections).
+ * awq_w4a16_linear -- step a7, the AWQ W4A16 linear (Diffusers blog, "From
+ * SVDQuant to Nunchaku Lite": awq_w4a16 for the memory-bound adaptive-norm
+ * modulation projections; int4 weights, a bf16 scale and zero point per 64
+ * values along K, 16-bit activations).
  *
  *   Y[m,n] = sum_k X[m,k] (q[n,k] - z[n,k/64]) s[n,k/64] + bias[n]
  *
- * X        device, bf16 [M, K] (row-major, K contiguous), 1 <= M <= 64; launches
- *          cover up to 16 tokens each (fewer when K is large)
+ * Two kernels serve it, by M: up to 64 tokens a GEMV on the warp-level MMA
+ * (launches of at most 16 tokens, each streaming the weights once); above 64 a
+ * tensor-core GEMM (tcgen05, tokens in tiles of up to 128, each tile streaming
+ * the weights once). Both form (q - z) exactly in bf16 and scale each group's
+ * float32 sum by s in float32. SVDQ_AWQ_PATH=0 / 1 in the environment forces the
+ * GEMV (M <= 64 only) / the GEMM for any M, for measurement.
+ *
+ * X        device, bf16 [M, K] (row-major, K contiguous), M >= 1
  * qweight  device, awq_qweight_bytes(N, K) bytes, fragment order from svdq_pack(AWQ)
- * sz       device, awq_sz_bytes(N, K) bytes, interleaved (s, z) from svdq_pack(AWQ)
+ * sz       device, awq_sz_bytes(N, K) bytes, interleaved (s, z) from svdq_pack(AWQ);
+ *          every zero point z is an integer in [0, 15], as the format defines
  * bias     device, bf16 [N] or NULL
  * Y        device, bf16 [M, N]
- * group must be 64. Accumulation is float32; (q - z) is exact in bf16 and each
- * group's sum is scaled by s in float32.
+ * group must be 64; INVALID_ARG / ALIGNMENT otherwise.
  */
 svdq_status awq_w4a16_linear(int M, int N, int K, int group, const void* X, const void* qweight,
                              const void* sz, const void* bias, void* Y, svdq_stream_t stream);
@@ -322,6 +379,66 @@ svdq_status svdq_unpack(svdq_pack_kind kind, svdq_format format, int rows, int K
  */
 svdq_status svdq_pack_lowrank(int K, int r, const void* L1, const float* smooth_inv, void* L1s,
                               svdq_stream_t stream);
+
+/*
+ * Offline weight preparation (Nunchaku README, "Method": stage 2 migrates the
+ * activation outliers into the weights, X_hat = X diag(lambda)^-1 and
+ * W_hat = W diag(lambda); stage 3 splits W_hat into a 16-bit low-rank part L1 L2
+ * and a residual R that is quantized to 4 bits). These calls run everything of
+ * it except the SVD, which the caller's linear-algebra library computes from
+ * W_hat = W diag(1 / smooth_inv) (in float64). Not part of the timed path.
+ *
+ * svdq_column_absmax -- absmax[k] = max_m |A[m,k]| (exact) of a bf16 matrix.
+ *   A       device, bf16 [rows, lda], 16-byte aligned, lda % 8 == 0, lda >= K
+ *   absmax  device, float32 [K], written (cleared first on the stream)
+ *   K % 8 == 0.
+ *
+ * svdq_smoothing -- the smoothing vector of one layer from the calibration
+ * activations' channel maxima and the weight:
+ *   lambda_k = sqrt(x_absmax[k] / max_n |W[n,k]|) in float64 (1 if either is 0),
+ *   smooth_inv[k] = RN32(1 / lambda_k) in float64, then rounded once to float32
+ *   x_absmax    device, float32 [K] (e.g. svdq_column_absmax of calibration X)
+ *   W           device, bf16 [N, K], 16-byte aligned
+ *   smooth_inv  device, float32 [K], written
+ *
+ * svdq_lowrank_factors -- the 16-bit low-rank factors from the SVD
+ * W_hat = U diag(S) Vh (float64, singular values in decreasing order), each
+ * element rounded once to bf16 (nearest even):
+ *   L1[k,j] = RN_bf16(Vh[j,k] sqrt(S[j]))  [K, r],   L2[j,n] = RN_bf16(sqrt(S[j]) U[n,j])  [r, N]
+ *   U [N, ldu] (ldu >= r), S [>= r], Vh [>= r rows, ldvh] (ldvh >= K): device, float64
+ *   L1, L2      device, bf16, written;  1 <= r <= min(N, K).
+ *
+ * svdq_residual -- the residual that is quantized:
+ *   R[n,k] = RN_bf16( W[n,k] * (1 / smooth_inv[k]) - sum_j L1[k,j] L2[j,n] ),
+ *   each step in float64, one rounding to bf16 (nearest even) at the end
+ *   W           device, bf16 [N, K];  smooth_inv  device, float32 [K]
+ *   L1, L2      device, bf16 [K, r] and [r, N] (the SVD factors); NULL iff r == 0
+ *   R           device, bf16 [N, K], written (quantize it with svdq_quantize_act,
+ *               no smoothing, rank 0)
+ *   0 <= r <= 4096.
+ *
+ * awq_quantize_weight -- the AWQ W4A16 weight quantizer (Diffusers blog,
+ * quantization_config: awq_w4a16, int4, group 64), per row and 64-wide group:
+ *   s = RN_bf16((max - min) / 15), or 1 if max == min;  z = clamp(rint(-min / s), 0, 15);
+ *   q = clamp(rint(w / s + z), 0, 15)   (float64 arithmetic, rint to even)
+ * written straight into the layouts awq_w4a16_linear reads (the output of
+ * svdq_pack(AWQ)).
+ *   W        device, bf16 [N, K]
+ *   qweight  device, awq_qweight_bytes(N, K) bytes, written
+ *   sz       device, awq_sz_bytes(N, K) bytes, written
+ *   K % 64 == 0.
+ * All five: INVALID_ARG / ALIGNMENT on bad arguments, before any launch.
+ */
+svdq_status svdq_column_absmax(int rows, int K, const void* A, int lda, float* absmax,
+                               svdq_stream_t stream);
+svdq_status svdq_smoothing(int N, int K, const float* x_absmax, const void* W, float* smooth_inv,
+                           svdq_stream_t stream);
+svdq_status svdq_lowrank_factors(int N, int K, int r, const double* U, int ldu, const double* S,
+                                 const double* Vh, int ldvh, void* L1, void* L2, svdq_stream_t stream);
+svdq_status svdq_residual(int N, int K, int r, const void* W, const float* smooth_inv, const void* L1,
+                          const void* L2, void* R, svdq_stream_t stream);
+svdq_status awq_quantize_weight(int N, int K, const void* W, void* qweight, void* sz,
+                                svdq_stream_t stream);
 
 /*
  * svdq_check_device_status -- synchronises `stream`, then reads and clears the

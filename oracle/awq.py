@@ -8,7 +8,7 @@ activations and 4-bit weights, ``precision: int4, group_size: 64``.
 
 Reading (asymmetric, the usual AWQ form): per group of 64 weights along K,
     s = BF16((max - min) / 15), s = 1 if max == min
-    z = clamp(rint(-min / s), 0, 15)            (an integer, exact in bf16)
+    z = clamp(rint(-min / s), 0, 15)            (an integer, exact in bf16; zero is +0)
     q = clamp(rint(w / s + z), 0, 15)
 and the layer computes y[m, n] = sum_k x[m, k] (q[n, k] - z[n, g]) s[n, g] + b[n].
 The activation-aware scale search needs calibration data and is not part of it.
@@ -30,7 +30,7 @@ def quantize_weight(w: np.ndarray):
     g = w.reshape(N, K // GROUP, GROUP)
     mx, mn = g.max(axis=2), g.min(axis=2)
     s = np.where(mx == mn, 1.0, bf16_round((mx - mn) / 15.0))
-    z = np.clip(np.rint(-mn / s), 0, 15)
+    z = np.clip(np.rint(-mn / s), 0, 15) + 0.0  # an integer: a zero point of zero is +0
     q = np.clip(np.rint(g / s[:, :, None] + z[:, :, None]), 0, 15)
     return q.reshape(N, K).astype(np.uint8), s, z
 

@@ -48,6 +48,11 @@ def svd_split(w_hat: np.ndarray, r: int):
     return L1, L2
 
 
+def residual(w_hat: np.ndarray, L1: np.ndarray, L2: np.ndarray) -> np.ndarray:
+    """R = W_hat - (L1 L2)^T, rounded once to bfloat16."""
+    return bf16_round(w_hat - (L1 @ L2).T)
+
+
 def prepare_svdq_layer(fmt: str, x_bits: np.ndarray, w_bits: np.ndarray, r: int) -> dict:
     """Everything the runtime layer needs, from bf16 X (calibration) and W."""
     x = bf16_from_bits(x_bits)
@@ -55,7 +60,7 @@ def prepare_svdq_layer(fmt: str, x_bits: np.ndarray, w_bits: np.ndarray, r: int)
     lam, smooth_inv = smoothing_factors(x, w)
     w_hat = w * (1.0 / smooth_inv)[None, :]
     L1, L2 = svd_split(w_hat, r)
-    R = bf16_round(w_hat - (L1 @ L2).T)
+    R = residual(w_hat, L1, L2)
     w_codes, w_scales = quantize(fmt, R)
     return {"lambda": lam, "smooth_inv": smooth_inv, "w_hat": w_hat, "L1": L1, "L2": L2,
             "R": R, "w_codes": w_codes, "w_scales": w_scales}

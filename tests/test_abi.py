@@ -85,7 +85,8 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert qkv(384, cos=odd, sin=good) == 2 and qkv(384, cos=good, sin=odd) == 2
     assert qkv(384, norm_q=P(0x10001)) == 2
     a = lib.awq_w4a16_linear
-    assert a(65, 16, 64, 64, good, good, good, None, good, None) == 1
+    assert a(0, 16, 64, 64, good, good, good, None, good, None) == 1     # M >= 1 (any M above)
+    assert a(4, 16, 96, 64, good, good, good, None, good, None) == 1     # K % 64
     assert a(4, 16, 64, 32, good, good, good, None, good, None) == 1
     assert a(4, 16, 64, 64, odd, good, good, None, good, None) == 2
     assert lib.svdq_pack(0, 0, 10, 64, good, good, good, good, good, None) == 1  # zeros for ACT

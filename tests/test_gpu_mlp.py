@@ -1,0 +1,140 @@
+"""The fused MLP (svdq_mlp_fc1, then svdq_w4a4_linear as fc2) against the oracle's
+fused MLP (oracle/mlp_epilogue.py) on the same seeded layers.
+
+The oracle forms h_hat from fc1's exact output in float64; the kernel from its
+float32 accumulator with a float32 GELU, so the two h_hat differ by a few float32
+roundings. The test therefore reads the kernel's h_hat back (the call's debug
+output) and checks: h_hat within that bound of the oracle's; fc2's codes and
+scales bit for bit against the oracle's quantizer applied to the kernel's h_hat;
+xl1_2 within the down-projection's error bound of the oracle's h_hat_kernel L1_2;
+fc2's output within the stated GEMM tolerance of the oracle's fc2 on that input;
+and within the stated relative L2 error of the oracle's whole fused MLP (an
+h_hat a few float32 roundings away can round to the neighbouring 4-bit code,
+which moves single outputs by a quantization step: the max-abs clause belongs
+to the GEMM given its input, not to a comparison across that rounding).
+Cases: units of one and of several tiles (the xl1_2 accumulator carried across
+tiles and added over several units), ragged M, r1 = 0 and r2 = 0, r2 = 128, and
+the FLUX-like MLP pair at full size on sampled rows."""
+
+import numpy as np
+import pytest
+
+import workloads as WL
+from oracle import formats as F
+from oracle import layout as LO
+from oracle import mlp_epilogue as E
+from oracle import prep as P
+from oracle import svdq as S
+from tests import svdq_cases as C
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_quantized_diffusion_b200 as bq
+    return bq
+
+
+def _layers(M, K1, N1, N2, r1, r2, seed):
+    """fc1 [N1, K1] and fc2 [N2, N1] layers, each prepared by the oracle from its
+    own seeded calibration activations (fc2's from an independent draw)."""
+    s1 = WL.custom_svdq("fc1", M, K1, N1, r1, seed=seed, n_outliers=4, outlier_scale=30.0,
+                        spike_rank=4, spike_sv=2.0)
+    s2 = WL.custom_svdq("fc2", M, N1, N2, r2, seed=seed + 1, n_outliers=4, outlier_scale=8.0,
+                        spike_rank=4, spike_sv=2.0)
+    d1, d2 = WL.svdq_inputs(s1), WL.svdq_inputs(s2)
+    p1 = P.prepare_svdq_layer("nvfp4", d1["X"], d1["W"], r1)
+    p2 = P.prepare_svdq_layer("nvfp4", d2["X"], d2["W"], r2)
+    return d1, p1, d2, p2
+
+
+def _run(bq, d1, p1, d2, p2, M, K1, N1, N2, r1, r2, with_hhat=True):
+    X = C.bf16_tensor(d1["X"][:M])
+    si1 = C.f32_tensor(p1["smooth_inv"])
+    L1s1 = bq.svdq_pack_lowrank(C.bf16_tensor(F.bf16_bits(p1["L1"])), si1) if r1 else None
+    a_c, a_s, xl1 = bq.svdq_quantize_act(X, L1s1, si1)
+    w1c, w1s, _ = bq.svdq_quantize_act(C.bf16_tensor(F.bf16_bits(p1["R"])), None, None)
+    w2c, w2s, _ = bq.svdq_quantize_act(C.bf16_tensor(F.bf16_bits(p2["R"])), None, None)
+    L2_1 = C.bf16_tensor(F.bf16_bits(p1["L2"])) if r1 else None
+    L1t_2 = C.bf16_tensor(F.bf16_bits(np.ascontiguousarray(p2["L1"].T))) if r2 else None
+    hhat = torch.empty((M, N1), dtype=torch.float32, device="cuda") if with_hhat else None
+    c2, s2, x2 = bq.svdq_mlp_fc1(a_c, a_s, xl1, w1c, w1s, L2_1, C.bf16_tensor(d1["bias"]),
+                                 C.f32_tensor(p2["smooth_inv"]), L1t_2, M, N1, K1, hhat=hhat)
+    L2_2 = C.bf16_tensor(F.bf16_bits(p2["L2"])) if r2 else None
+    y2 = bq.svdq_w4a4_linear(c2, s2, x2, w2c, w2s, L2_2, C.bf16_tensor(d2["bias"]), M, N2, N1)
+    assert bq.svdq_check_device_status() == 0
+    return {"codes2": c2, "scales2": s2, "xl1_2": x2, "hhat": hhat, "Y2": y2}
+
+
+def _check(bq, out, d1, p1, d2, p2, M, r2, rows=None):
+    rows = np.arange(M) if rows is None else rows
+    # the oracle: fc1's exact output, then the fused epilogue and fc2
+    y1 = S.svdq_forward("nvfp4", d1["X"][rows], p1["smooth_inv"], p1["L1"], p1["L2"],
+                        p1["w_codes"], p1["w_scales"], d1["bias"])["Y"]
+    ref = E.mlp_forward(y1, p2["smooth_inv"], p2["L1"], p2["L2"], p2["w_codes"], p2["w_scales"],
+                        F.bf16_from_bits(d2["bias"]))
+    hk = out["hhat"].cpu().numpy().astype(np.float64)[rows]
+    ho = ref["h_hat"]
+    bound = 2.0 ** -13 * np.sqrt(np.mean(ho ** 2)) + 2.0 ** -16 * np.abs(ho)
+    worst = np.unravel_index(np.argmax(np.abs(hk - ho) - bound), hk.shape)
+    assert np.all(np.abs(hk - ho) <= bound), (
+        f"h_hat at {worst}: kernel {hk[worst]}, oracle {ho[worst]}")
+    # fc2's input, bit for bit against the oracle's quantizer on the kernel's h_hat
+    q, sc = S.quantize("nvfp4", hk)
+    N1 = hk.shape[1]
+    codes = out["codes2"].cpu().numpy().reshape(M, N1 // 2)[rows]
+    assert np.array_equal(codes, S.pack_nibbles(q))
+    tiled = out["scales2"].cpu().numpy()
+    full = LO.untile_nvfp4_scales(tiled, M, N1)
+    assert np.array_equal(full[rows], sc)
+    if r2:
+        xk = out["xl1_2"].cpu().numpy().astype(np.float64)[rows]
+        xo = S.down_proj(hk, p2["L1"])
+        assert np.all(np.abs(xk - xo) <= C.xl1_bound(hk, p2["L1"]))
+    y2 = out["Y2"].float().cpu().numpy().astype(np.float64)[rows]
+    # fc2 on exactly the input the fused epilogue produced: the full GEMM tolerance
+    xl1_k = out["xl1_2"].cpu().numpy().astype(np.float64)[rows] if r2 else None
+    y2_ref = S.w4a4_linear(S.dequant_nvfp4(q, sc), S.dequant_nvfp4(p2["w_codes"], p2["w_scales"]),
+                           xl1_k, p2["L2"] if r2 else None, F.bf16_from_bits(d2["bias"]))
+    C.assert_gemm_close(y2, y2_ref, bf16_out=True, what="fc2 Y on the fused epilogue's output")
+    # and the whole MLP against the oracle's, from fc1's exact output: an h_hat a few
+    # float32 roundings away may sit on the other side of a 4-bit rounding boundary,
+    # which moves single outputs by a quantization step, so only the relative L2
+    # error is bounded here
+    rl = C.rel_l2(y2, ref["Y"])
+    assert rl <= 2e-3, f"fused MLP: rel-L2 {rl:.3e} against the oracle's MLP"
+
+
+@pytest.mark.parametrize("M,K1,N1,N2,r1,r2", [
+    (300, 512, 512, 256, 32, 32),      # one tile per unit, ragged rows
+    (1300, 512, 1536, 384, 32, 64),    # several tiles per unit, xl1_2 carried across them
+    (200, 1024, 384, 128, 64, 128),    # the largest r2
+    (100, 256, 256, 128, 0, 0),        # no low-rank branch on either side
+])
+def test_fused_mlp_matches_the_oracle(bq, M, K1, N1, N2, r1, r2):
+    d1, p1, d2, p2 = _layers(M, K1, N1, N2, r1, r2, seed=50 + r2 + M)
+    out = _run(bq, d1, p1, d2, p2, M, K1, N1, N2, r1, r2)
+    _check(bq, out, d1, p1, d2, p2, M, r2)
+    # without the h_hat read-back the call writes the same bytes
+    again = _run(bq, d1, p1, d2, p2, M, K1, N1, N2, r1, r2, with_hhat=False)
+    for k in ("codes2", "scales2") + (("xl1_2",) if r2 else ()):
+        assert torch.equal(again[k].view(torch.uint8), out[k].view(torch.uint8)), k
+
+
+@pytest.mark.slow
+def test_fused_mlp_full_size_sampled(bq):
+    """The FLUX-like MLP pair (fc1 4608 x 3072 -> 12288, fc2 12288 -> 3072, rank 128) in
+    the launch configuration the benchmark times, checked on six 128-row blocks."""
+    s1, s2 = WL.FC1, WL.FC2
+    d1, d2 = WL.svdq_inputs(s1), WL.svdq_inputs(s2)
+    p1 = P.prepare_svdq_layer("nvfp4", d1["X"], d1["W"], s1.r)
+    p2 = P.prepare_svdq_layer("nvfp4", d2["X"], d2["W"], s2.r)
+    M = s1.M
+    out = _run(bq, d1, p1, d2, p2, M, s1.K, s1.N, s2.N, s1.r, s2.r)
+    blocks = np.unique(np.linspace(0, (M + 127) // 128 - 1, 6).round().astype(int))
+    rows = np.concatenate([np.arange(b * 128, min(M, b * 128 + 128)) for b in blocks])
+    _check(bq, out, d1, p1, d2, p2, M, s2.r, rows=rows)

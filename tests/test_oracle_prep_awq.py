@@ -60,6 +60,10 @@ def test_awq_quantize_properties():
     q, s, z = A.quantize_weight(w)
     assert q.min() >= 0 and q.max() <= 15
     assert np.array_equal(F.bf16_round(s), s) and np.all(z == np.rint(z))
+    assert not np.any(np.signbit(z))  # integer zero points: a zero is +0
+    # a constant positive group: s = 1, rint(-min) = -0 becomes the integer +0
+    qc, sc, zc = A.quantize_weight(np.full((1, 64), 0.125))
+    assert sc[0, 0] == 1.0 and zc[0, 0] == 0.0 and not np.signbit(zc[0, 0]) and not qc.any()
     deq = A.dequant_weight(q, s, z)
     # codes strictly inside (0, 15) come from rint: error at most half a step
     sv = np.repeat(s, 64, axis=1)
