@@ -133,7 +133,7 @@ def sweep_layers(bq, prep, dev, flush, n: int, fp4_peak: float) -> dict:
         X = to_dev(d["X"])
         W = to_dev(d["W"])
         bias = to_dev(d["bias"]) if d["bias"] is not None else None
-        x_absmax = X.float().abs().amax(dim=0)
+        x_absmax = bq.svdq_column_absmax(X)
         svd = None
         if sh.r > 0:
             key = (sh.seed, sh.N, sh.K)
@@ -177,6 +177,75 @@ def sweep_layers(bq, prep, dev, flush, n: int, fp4_peak: float) -> dict:
                 (e["svdq_w4a4_linear_us"] + e["svdq_quantize_act_us"])
                 / (base["svdq_w4a4_linear_us"] + base["svdq_quantize_act_us"]) - 1, 3)
     return out
+
+
+def mlp_pair(bq, prep, dev, flush, n: int) -> dict:
+    """The FLUX-like MLP pair (fc1 4608 x 3072 -> 12288, GELU, fc2 12288 -> 3072, rank 128,
+    NVFP4), fused and unfused, each timed as a whole (event to event after the flush).
+    Unfused: quantizer, fc1 GEMM to bf16, GELU (tanh form, torch, bf16), fc2's quantizer
+    on that bf16 activation, fc2 GEMM. Fused: quantizer, svdq_mlp_fc1 (GELU, fc2's
+    smoothing, codes, scales and down-projection in fc1's epilogue, plus the reduction
+    of its partial down-projections), fc2 GEMM."""
+    import torch
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    s1, s2 = WL.FC1, WL.FC2
+    d1, d2 = WL.svdq_inputs(s1), WL.svdq_inputs(s2)
+    X1, X2c = to_dev(d1["X"]), to_dev(d2["X"])
+    ws = []
+    for d, sh, X in ((d1, s1, X1), (d2, s2, X2c)):
+        W = to_dev(d["W"])
+        xa = bq.svdq_column_absmax(X)
+        _, w_hat = prep.smoothed_weight(W, xa)
+        svd = torch.linalg.svd(w_hat.float(), full_matrices=False)
+        ws.append(prep.prepare_svdq_weights(W, xa, sh.r, svd=svd))
+        del W, w_hat, svd
+    w1, w2 = ws
+    del X2c
+    b1, b2 = to_dev(d1["bias"]), to_dev(d2["bias"])
+    M, K1, N1, N2, r1, r2 = s1.M, s1.K, s1.N, s2.N, s1.r, s2.r
+    L1t_2 = w2["L1"].t().contiguous()
+    c1 = torch.empty(bq.svdq_codes_bytes("nvfp4", M, K1), dtype=torch.uint8, device=dev)
+    sc1 = torch.empty(bq.svdq_scales_bytes("nvfp4", M, K1), dtype=torch.uint8, device=dev)
+    x1 = torch.empty((bq.svdq_xl1_splits(M, K1, r1), M, r1), dtype=torch.float32, device=dev)
+    c2 = torch.empty(bq.svdq_codes_bytes("nvfp4", M, N1), dtype=torch.uint8, device=dev)
+    sc2 = torch.empty(bq.svdq_scales_bytes("nvfp4", M, N1), dtype=torch.uint8, device=dev)
+    x2f = torch.empty((bq.svdq_mlp_splits(M, N1), M, r2), dtype=torch.float32, device=dev)
+    x2u = torch.empty((bq.svdq_xl1_splits(M, N1, r2), M, r2), dtype=torch.float32, device=dev)
+    Y1 = torch.empty((M, N1), dtype=torch.bfloat16, device=dev)
+    Y2 = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+
+    def quant1():
+        return bq.svdq_quantize_act(X1, w1["L1s"], w1["smooth_inv"], codes=c1, scales=sc1, xl1=x1)[2]
+
+    def unfused():
+        xv = quant1()
+        bq.svdq_w4a4_linear(c1, sc1, xv, w1["w_codes"], w1["w_scales"], w1["L2"], b1, M, N1, K1, Y=Y1)
+        h = torch.nn.functional.gelu(Y1, approximate="tanh")
+        _, _, xv2 = bq.svdq_quantize_act(h, w2["L1s"], w2["smooth_inv"], codes=c2, scales=sc2, xl1=x2u)
+        bq.svdq_w4a4_linear(c2, sc2, xv2, w2["w_codes"], w2["w_scales"], w2["L2"], b2, M, N2, N1, Y=Y2)
+
+    def fused_fc1():
+        xv = quant1()
+        return bq.svdq_mlp_fc1(c1, sc1, xv, w1["w_codes"], w1["w_scales"], w1["L2"], b1, w2["smooth_inv"],
+                               L1t_2, M, N1, K1, codes2=c2, scales2=sc2, xl1_2=x2f)[2]
+
+    def fused():
+        xv2 = fused_fc1()
+        bq.svdq_w4a4_linear(c2, sc2, xv2, w2["w_codes"], w2["w_scales"], w2["L2"], b2, M, N2, N1, Y=Y2)
+
+    xv = quant1()
+    t = {"unfused_us": median_us(unfused, flush, n), "fused_us": median_us(fused, flush, n),
+         "fused_fc1_us": median_us(lambda: bq.svdq_mlp_fc1(
+             c1, sc1, xv, w1["w_codes"], w1["w_scales"], w1["L2"], b1, w2["smooth_inv"], L1t_2, M, N1, K1,
+             codes2=c2, scales2=sc2, xl1_2=x2f), flush, n)}
+    assert bq.svdq_check_device_status() == 0
+    flops = 2.0 * M * N1 * K1 + 2.0 * M * N2 * N1
+    return {"workload": f"{s1.name} -> GELU -> {s2.name}: M={M} K1={K1} N1={N1} N2={N2} r={r1}",
+            **{k: round(v, 2) for k, v in t.items()},
+            "fused_speedup": round(t["unfused_us"] / t["fused_us"], 3),
+            "fused_fc1_tflops_4bit": round(2.0 * M * N1 * K1 / (t["fused_fc1_us"] * 1e-6) / 1e12, 1),
+            "fused_pair_tflops_4bit": round(flops / (t["fused_us"] * 1e-6) / 1e12, 1),
+            "hidden_bytes_avoided": 2 * M * N1 * 2}
 
 
 def awq_by_tokens(bq, awq_w, bias_a, dev, flush, n: int) -> dict:
@@ -521,7 +590,7 @@ def main() -> None:
     X = to_dev(x_bits)
     W = to_dev(d["W"])
     bias = to_dev(d["bias"])
-    x_absmax = X.float().abs().amax(dim=0)
+    x_absmax = bq.svdq_column_absmax(X)
     svdq_w = prep.prepare_svdq_weights(W, x_absmax, SHAPE.r, "nvfp4")
     da = WL.awq_inputs(AWQ)
     Xa = to_dev(da["X"])
@@ -649,12 +718,13 @@ def main() -> None:
     status = status or bq.svdq_check_device_status()
 
     # ------------------------------- the other workloads and AWQ at more tokens
-    sweep, awq_tokens = None, None
+    sweep, awq_tokens, mlp = None, None, None
     if not args.no_sweep and rank == 0:
         peaks0 = measured_peaks()
         sweep = sweep_layers(bq, prep, dev, flush, max(3, min(args.steps, 50)),
                              peaks0["bf16_tflops"] * FP4_OVER_BF16)
         awq_tokens = awq_by_tokens(bq, awq_w, bias_a, dev, flush, max(3, min(args.steps, 50)))
+        mlp = mlp_pair(bq, prep, dev, flush, max(3, min(args.steps, 50)))
 
     # ----------------------------------------------- end to end, host buffers
     Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
@@ -806,6 +876,8 @@ def main() -> None:
             "timing": "each layer's quantizer and GEMM called alone after the L2 flush, event to event, "
                       "median of the calls",
             **sweep}
+        out["kernels"]["fused_mlp"] = {
+            "timing": "the whole MLP pair per call, event to event after the flush, median", **mlp}
         out["kernels"]["awq_by_tokens"] = {
             "timing": f"awq_w4a16_linear at K={AWQ.K} N={AWQ.N}, event to event after the flush, median; "
                       f"the GEMV (warp-level MMA) serves M <= 64, the tensor-core GEMM any M",

@@ -5,7 +5,8 @@
 // activation never reaches HBM in 16 bits:
 //
 //   y1     = Q(X1_hat) Q(R1)^T + xl1_1 L2_1 + bias1                (tensor memory, float32)
-//   h_hat  = RN32(RN32(GELU_tanh(RN32(y1))) * smooth_inv2[n])      (epilogue, float32)
+//   h_hat  = RN32(RN32(GELU_tanh(RN32(y1))) * smooth_inv2[n])      (epilogue, float32; GELU as
+//            y / (1 + exp(-2u)), which equals its tanh form 0.5 y (1 + tanh(u)), to a few ulps)
 //   codes2, scales2 = NVFP4 of h_hat, groups of 16 along N1         (fc2's tiled layouts)
 //   xl1_2  = h_hat L1_2                                            (tensor cores, float32)
 //
@@ -83,10 +84,19 @@ struct MlpParams {
   uint32_t* status;
 };
 
-// 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) in float32
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float u = 0.7978845608028654f * __fmaf_rn(0.044715f * y, y * y, y);
-  return 0.5f * y * (1.0f + tanhf(u));
+// GELU of two values: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3), in
+// float32 through the identity 1 + tanh(u) = 2 / (1 + exp(-2u)), i.e. GELU =
+// y / (1 + exp(-2u)): one exponential and one division per value (a few float32
+// ulps), the polynomial on paired float32 instructions. The form has no
+// cancellation; exp's argument is capped at 80 (finite in float32), where GELU
+// is 0 to float32 precision already.
+__device__ __forceinline__ float2 gelu_tanh2(float2 y) {
+  const float2 yy = __fmul2_rn(y, y);
+  const float2 a = __fmul2_rn(y, make_float2(0.044715f, 0.044715f));
+  const float2 t = __ffma2_rn(a, yy, y);                                         // y + 0.044715 y^3
+  const float2 m = __fmul2_rn(t, make_float2(-1.5957691216057308f, -1.5957691216057308f));  // -2u
+  const float dx = 1.0f + __expf(fminf(m.x, 80.0f)), dy = 1.0f + __expf(fminf(m.y, 80.0f));
+  return make_float2(__fdividef(y.x, dx), __fdividef(y.y, dy));
 }
 
 __global__ void __launch_bounds__(kMlThreads, 1)
@@ -466,10 +476,13 @@ __global__ void __launch_bounds__(kMlThreads, 1)
           }
           float hv[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float y = __fadd_rn(__uint_as_float(acc[q]), stg[32 * t + q]);
-            const float h = gelu_tanh(y);
-            hv[q] = m_ok ? __fmul_rn(h, stg[64 + 32 * t + q]) : 0.0f;
+          for (int q = 0; q < 32; q += 2) {
+            const float2 b = *reinterpret_cast<const float2*>(stg + 32 * t + q);
+            const float2 sm = *reinterpret_cast<const float2*>(stg + 64 + 32 * t + q);
+            const float2 y = __fadd2_rn(make_float2(__uint_as_float(acc[q]), __uint_as_float(acc[q + 1])), b);
+            const float2 h = __fmul2_rn(gelu_tanh2(y), sm);
+            hv[q] = m_ok ? h.x : 0.0f;
+            hv[q + 1] = m_ok ? h.y : 0.0f;
           }
           if (p.hhat != nullptr && m_ok) {
             float4* dst = reinterpret_cast<float4*>(p.hhat + static_cast<size_t>(m) * N1 + n0 + j0);
@@ -488,10 +501,11 @@ __global__ void __launch_bounds__(kMlThreads, 1)
             const float sv = e4m3_value(sc[g]);
             const float rcp = sv != 0.0f ? __frcp_rn(sv) : 0.0f;
             float2 y0[4], y1[4];
+            const float2 rcp2 = make_float2(rcp, rcp);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              y0[q] = make_float2(__fmul_rn(pv[q].x, rcp), __fmul_rn(pv[q].y, rcp));
-              y1[q] = make_float2(__fmul_rn(pv[4 + q].x, rcp), __fmul_rn(pv[4 + q].y, rcp));
+              y0[q] = __fmul2_rn(pv[q], rcp2);
+              y1[q] = __fmul2_rn(pv[4 + q], rcp2);
             }
             code[2 * g] = sv != 0.0f ? e2m1x8(y0) : 0u;
             code[2 * g + 1] = sv != 0.0f ? e2m1x8(y1) : 0u;
@@ -517,10 +531,10 @@ __global__ void __launch_bounds__(kMlThreads, 1)
               uint32_t hi[4], lo[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float x0 = hv[8 * cc + 2 * j], x1 = hv[8 * cc + 2 * j + 1];
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-                const float2 hf = __bfloat1622float2(hb);
-                const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+                const float2 x = make_float2(hv[8 * cc + 2 * j], hv[8 * cc + 2 * j + 1]);
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
+                const float2 r = __fadd2_rn(x, make_float2(-__bfloat162float(hb.x), -__bfloat162float(hb.y)));
+                const __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
                 hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
                 lo[j] = *reinterpret_cast<const uint32_t*>(&lb);
               }

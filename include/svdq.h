@@ -256,7 +256,8 @@ svdq_status svdq_w4a4_linear_two_level(int M, int N, int K, int r, const void* a
  *
  *   y1     = the fc1 layer as svdq_w4a4_linear computes it, float32 in tensor memory
  *   h_hat  = RN32(RN32(GELU(RN32(y1))) * smooth_inv2[n]),
- *            GELU(y) = 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) in float32
+ *            GELU(y) = 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3), evaluated in
+ *            float32 as y / (1 + exp(-2u)) (the same function; a few float32 ulps)
  *   codes2, scales2 = NVFP4 codes and scales of h_hat (steps a2, a3 of fc2, groups of 16
  *            along N1, the layouts svdq_quantize_act writes)
  *   xl1_2  = h_hat L1_2 (step a4 of fc2; h_hat as a bf16 hi + lo pair on the tensor
