@@ -110,8 +110,12 @@ def svdq_quantize_act_noalloc(X: torch.Tensor, L1s: torch.Tensor | None = None,
                               smooth_inv: torch.Tensor | None = None, fmt="nvfp4",
                               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
                               xl1: torch.Tensor | None = None, stream=None):
-    """svdq_quantize_act with xl1 only [M, r]: the library's static device array
-    holds the K splits' partial sums (see include/svdq.h for the limit)."""
+    """svdq_quantize_act with xl1 only [M, r] and no working space from the caller,
+    for callers whose allocator cannot grant memory mid-step (a runtime or plugin
+    that sized all device memory up front): the K splits' partial sums go to one
+    static device array the library holds per device, (S - 1) * M * r <= 2^21
+    floats; larger requests raise SvdqError. Two such calls that overlap on the
+    GPU race on that array."""
     lib = N.load()
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bf16 tensor")

@@ -1,7 +1,11 @@
 """svdq_quantize_act_noalloc against svdq_quantize_act on the GPU.
 
-The allocation-free entry point keeps the K splits' partial down-projections
-in a static device array instead of the caller's workspace; on the same inputs
+The allocation-free entry point is for callers that cannot hand the library
+working memory: a serving runtime or a plugin whose allocator sized all device
+memory before the first request, where an allocation mid-step would escape that
+budget, could block or synchronise the device, and could fail under memory
+pressure. It keeps the K splits' partial down-projections in a static device
+array instead of the caller's workspace; on the same inputs
 it must return the same bytes as the regular call, on two calls in a row, each
 right after a call on another activation of the same shape (so every compared
 call finds the array holding someone else's partial sums). This file is
