@@ -22,7 +22,8 @@
 // Layout of the work: CTA pairs (cta_group::2), tiles of 256 rows x 128
 // columns (each CTA stages its 128 rows of A and 64 of the tile's 128 B rows).
 // Tensor memory per CTA: two 128-column fc1 accumulators (tile i uses i % 2),
-// the xl1_2 accumulator (128 columns), two 32-column scale-factor buffers.
+// the xl1_2 accumulator (128 columns), four 32-column scale-factor buffers (the
+// quadrant warps may fill a buffer once the MMAs four 4-bit slots back are done).
 // Ring slots of a unit, in order: for each tile its K/256 FP4 slots and
 // ceil(r1/32) low-rank slots, then (from the second tile on) the xl1_2 slot of
 // the previous tile (L1_2^T's [r2/2 x 128] slice per CTA); after the last tile
@@ -58,12 +59,14 @@ constexpr uint32_t kMlHhat = kMlStages * kMlStageBytes;            // [hi, lo][2
 constexpr uint32_t kMlHhatPlane = 2 * kMlBM * 128;                 // 32 KB
 constexpr uint32_t kMlStaging = kMlHhat + 2 * kMlHhatPlane;        // bias1, smooth_inv2 per epilogue warp
 constexpr uint32_t kMlBars = kMlStaging + 8 * 2 * 64 * 4;
-// full, empty, ready, sf landed per stage; acc full, acc free x2; sf full, sf free x2;
+// full, empty, ready, sf landed per stage; acc full, acc free x2; sf full, sf free x4;
 // hhat full, hhat free; xl1_2 full, xl1_2 free
-constexpr uint32_t kMlTmemSlot = kMlBars + 8 * (4 * kMlStages + 4 + 4 + 4);
+constexpr int kMlSfBufs = 4;                      // scale-factor buffers in tensor memory
+constexpr uint32_t kMlTmemSlot = kMlBars + 8 * (4 * kMlStages + 4 + 2 * kMlSfBufs + 4);
 constexpr size_t kMlSmemBytes = kMlTmemSlot + 16 + 1024;
 // tensor-memory columns
 constexpr uint32_t kMlTmAcc = 0, kMlTmXl1 = 256, kMlTmSf = 384, kMlTmSfBuf = 32, kMlTmCols = 512;
+static_assert(kMlTmSf + kMlSfBufs * kMlTmSfBuf <= kMlTmCols, "tensor-memory layout");
 static_assert(kMlStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
 static_assert(kMlLrBTile + 2 * kMlBM * kMlLrK * 2 <= kMlStageBytes, "a low-rank slot fits in a stage");
 static_assert(2 * (kMlR2Max / 2) * 128 <= kMlStageBytes, "an xl1_2 slot fits in a stage");
@@ -139,9 +142,9 @@ __global__ void __launch_bounds__(kMlThreads, 1)
   auto bar_acc_full = [&](int a) { return bar0 + 8 * a; };
   auto bar_acc_free = [&](int a) { return bar0 + 16 + 8 * a; };
   auto bar_sf_full = [&](int b) { return bar0 + 32 + 8 * b; };
-  auto bar_sf_free = [&](int b) { return bar0 + 48 + 8 * b; };
-  const uint32_t bar_hh_full = bar0 + 64, bar_hh_free = bar0 + 72;
-  const uint32_t bar_x2_full = bar0 + 80, bar_x2_free = bar0 + 88;
+  auto bar_sf_free = [&](int b) { return bar0 + 32 + 8 * kMlSfBufs + 8 * b; };
+  const uint32_t bar_hh_full = bar0 + 32 + 16 * kMlSfBufs, bar_hh_free = bar_hh_full + 8;
+  const uint32_t bar_x2_full = bar_hh_full + 16, bar_x2_free = bar_hh_full + 24;
   auto lead = [&](uint32_t a) { return map_peer_smem(a, 0); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMlTmemSlot);
 
@@ -155,8 +158,10 @@ __global__ void __launch_bounds__(kMlThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_acc_full(a), 1);
       mbar_init(bar_acc_free(a), 8 * 2);
-      mbar_init(bar_sf_full(a), 4 * 2);
-      mbar_init(bar_sf_free(a), 1);
+    }
+    for (int b = 0; b < kMlSfBufs; ++b) {
+      mbar_init(bar_sf_full(b), 4 * 2);
+      mbar_init(bar_sf_free(b), 1);
     }
     mbar_init(bar_hh_full, 8 * 2);
     mbar_init(bar_hh_free, 1);
@@ -273,8 +278,8 @@ __global__ void __launch_bounds__(kMlThreads, 1)
               int s;
               if (!take(s)) break;
               if (kt < ktiles) {
-                const uint32_t buf = static_cast<uint32_t>(fp4 & 1);
-                ok = mbar_wait(bar_sf_full(buf), (fp4 >> 1) & 1, p.status);
+                const uint32_t buf = static_cast<uint32_t>(fp4 % kMlSfBufs);
+                ok = mbar_wait(bar_sf_full(buf), (fp4 / kMlSfBufs) & 1, p.status);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sfa = tmem + kMlTmSf + kMlTmSfBuf * buf, sfb = sfa + 16;
@@ -359,7 +364,7 @@ __global__ void __launch_bounds__(kMlThreads, 1)
           for (int kt = 0; kt < ktiles && ok; ++kt, ++fp4) {
             int s;
             if (!wait_slot(s)) break;
-            const int buf = fp4 & 1;
+            const int buf = fp4 % kMlSfBufs;
             uint32_t sa[16], sbv[16];
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
@@ -368,7 +373,7 @@ __global__ void __launch_bounds__(kMlThreads, 1)
               const uint4 b = lds_u4(sfb_st(s) + kb * 512 + lane * 16);
               sbv[4 * kb] = b.x; sbv[4 * kb + 1] = b.y; sbv[4 * kb + 2] = b.z; sbv[4 * kb + 3] = b.w;
             }
-            ok = fp4 < 2 || mbar_wait(bar_sf_free(buf), ((fp4 >> 1) - 1) & 1, p.status);
+            ok = fp4 < kMlSfBufs || mbar_wait(bar_sf_free(buf), ((fp4 / kMlSfBufs) - 1) & 1, p.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();

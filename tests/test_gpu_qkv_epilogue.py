@@ -17,6 +17,7 @@ import pytest
 
 import workloads as WL
 from oracle import formats as F
+from oracle import layout as LO
 from oracle import qkv_epilogue as E
 from oracle import svdq as S
 from tests import svdq_cases as C
@@ -117,7 +118,8 @@ def test_unit_weights_give_unit_mean_square_heads(bq):
 @pytest.mark.slow
 def test_full_size_flux_qkv(bq):
     """M = 4608, K = 3072, N = 9216 (24 heads each), r = 32: weights from the
-    library's own prep, the bench's launch configuration."""
+    library's own prep, the bench's launch configuration; Q and K on six sampled
+    128-row blocks against the oracle's layer followed by its epilogue."""
     from bit_quantized_diffusion_b200 import prep
     shape = WL.QKV
     M, K, N, r, H = shape.M, shape.K, shape.N, shape.r, shape.N // (3 * D)
@@ -125,7 +127,7 @@ def test_full_size_flux_qkv(bq):
     X = C.bf16_tensor(d["X"])
     W = C.bf16_tensor(d["W"])
     bias = C.bf16_tensor(d["bias"])
-    w = prep.prepare_svdq_weights(W, X.float().abs().amax(dim=0), r, "nvfp4")
+    w = prep.prepare_svdq_weights(W, bq.svdq_column_absmax(X), r, "nvfp4")
     codes, scales, xl1 = bq.svdq_quantize_act(X, w["L1s"], w["smooth_inv"])
     ep = WL.qkv_epilogue_inputs(M, seed=90, angles="positions")
     gq, gk = C.bf16_tensor(ep["norm_q"]), C.bf16_tensor(ep["norm_k"])
@@ -140,10 +142,23 @@ def test_full_size_flux_qkv(bq):
     assert torch.equal(y[:, 2 * H * D:], plain[:, 2 * H * D:])
     blocks = np.unique(np.linspace(0, M // 128 - 1, 6).round().astype(int))
     rows = np.unique(np.concatenate([np.arange(b * 128, b * 128 + 128) for b in blocks] + [[M - 1]]))
-    ref = E.qkv_norm_rope(as_f64(plain32[rows]), H, F.bf16_from_bits(ep["norm_q"]),
-                          F.bf16_from_bits(ep["norm_k"]), 1e-6, ep["cos"][rows], ep["sin"][rows])
+    # the oracle's layer on those rows, with the weights the library prepared (in the
+    # oracle's plain formats), followed by the oracle's epilogue
+    bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+    w_codes = S.unpack_nibbles(w["w_codes"].cpu().numpy().reshape(N, K // 2))
+    w_scales = LO.untile_nvfp4_scales(w["w_scales"].cpu().numpy(), N, K)
+    fwd = S.svdq_forward("nvfp4", d["X"][rows], w["smooth_inv"].cpu().numpy().astype(np.float64),
+                         F.bf16_from_bits(bits(w["L1"])), F.bf16_from_bits(bits(w["L2"])), w_codes, w_scales,
+                         d["bias"])
+    ref = E.qkv_norm_rope(fwd["Y"], H, F.bf16_from_bits(ep["norm_q"]), F.bf16_from_bits(ep["norm_k"]), 1e-6,
+                          ep["cos"][rows], ep["sin"][rows])
     C.assert_gemm_close(as_f64(y[rows])[:, :2 * H * D], ref[:, :2 * H * D], bf16_out=True,
                         what="Q, K (full size)")
+    # and the plain call's float32 output through the same epilogue (the epilogue alone)
+    ref32 = E.qkv_norm_rope(as_f64(plain32[rows]), H, F.bf16_from_bits(ep["norm_q"]),
+                            F.bf16_from_bits(ep["norm_k"]), 1e-6, ep["cos"][rows], ep["sin"][rows])
+    C.assert_gemm_close(as_f64(y[rows])[:, :2 * H * D], ref32[:, :2 * H * D], bf16_out=True,
+                        what="Q, K against the plain call's epilogue")
 
 
 def test_layer_class_matches_the_oracle(bq):
