@@ -702,8 +702,8 @@ def main() -> None:
     # epilogue, timed event to event after the flush, against the plain GEMM above.
     qe = WL.qkv_epilogue_inputs(M, seed=SHAPE.seed + 100, angles="positions")
     norm_q, norm_k = to_dev(qe["norm_q"]), to_dev(qe["norm_k"])
-    rope_cos = torch.from_numpy(qe["cos"]).to(dev)
-    rope_sin = torch.from_numpy(qe["sin"]).to(dev)
+    rope_cos = torch.from_numpy(np.ascontiguousarray(qe["cos"].T)).to(dev)  # angle-major [64, M]
+    rope_sin = torch.from_numpy(np.ascontiguousarray(qe["sin"].T)).to(dev)
     Y3 = torch.empty_like(Y)
     ev3 = [[mk() for _ in range(2)] for _ in range(n2 + 3)]
     for i in range(n2 + 3):

@@ -242,7 +242,8 @@ def svdq_w4a4_linear_qkv_norm_rope(a_codes, a_scales, xl1, w_codes, w_scales, L2
     """The fused QKV projection (NVFP4): Y [M, N] = Q(X_hat) Q(R)^T + xl1 @ L2 + bias with
     every 128-column head of Q and K (columns [0, N/3) and [N/3, 2N/3)) RMS-normalised
     (norm_q / norm_k bf16 [128] or None, eps) and then turned pairwise by rope_cos /
-    rope_sin float32 [M, 64] (both None: no rotation); V unchanged. N % 384 == 0."""
+    rope_sin float32 [64, M], angle-major (angle i of row m at [i, m]; both None: no
+    rotation); V unchanged. N % 384 == 0."""
     lib = N.load()
     r = 0 if L2 is None else L2.shape[0]
     if r and (xl1 is None or xl1.dtype != torch.float32 or xl1.numel() < M * r):
@@ -260,9 +261,9 @@ def svdq_w4a4_linear_qkv_norm_rope(a_codes, a_scales, xl1, w_codes, w_scales, L2
         if g is not None and (g.dtype != torch.bfloat16 or g.numel() != 128 or not g.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous bf16 [128]")
     for tb, name in ((rope_cos, "rope_cos"), (rope_sin, "rope_sin")):
-        if tb is not None and (tb.dtype != torch.float32 or tuple(tb.shape) != (M, 64)
+        if tb is not None and (tb.dtype != torch.float32 or tuple(tb.shape) != (64, M)
                                or not tb.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous float32 [M, 64]")
+            raise ValueError(f"{name} must be a contiguous float32 [64, M] (angle-major)")
     f = N.NVFP4_G16
     _need(a_codes, lib.svdq_codes_bytes(f, M, K), "a_codes")
     _need(a_scales, lib.svdq_scales_bytes(f, M, K), "a_scales")

@@ -201,6 +201,7 @@ svdq_status device_setup(DeviceInfo** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool debug_on() { return std::getenv("SVDQ_DEBUG") != nullptr; }
 
@@ -669,7 +670,7 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(int M, int N, int K, int r, const voi
                                            void* Y, int ldy, svdq_out out, svdq_stream_t stream) {
   if (N < 384 || N % 384 || !(eps >= 0.0f) || eps > 3.0e38f) return SVDQ_ERR_INVALID_ARG;
   if ((rope_cos != nullptr) != (rope_sin != nullptr)) return SVDQ_ERR_INVALID_ARG;
-  if ((rope_cos && (!aligned16(rope_cos) || !aligned16(rope_sin))) ||
+  if ((rope_cos && (!aligned4(rope_cos) || !aligned4(rope_sin))) ||
       (reinterpret_cast<uintptr_t>(norm_q) & 1u) || (reinterpret_cast<uintptr_t>(norm_k) & 1u))
     return SVDQ_ERR_ALIGNMENT;
   const QkNormArgs qk{N / 384, eps, norm_q, norm_k, rope_cos, rope_sin};

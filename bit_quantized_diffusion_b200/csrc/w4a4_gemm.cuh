@@ -57,9 +57,12 @@
 // squares of its columns of each head (y = alpha acc + bias in float32), the two
 // trade their partial sums through shared memory behind a per-quadrant
 // mbarrier, and each then scales its columns by rsqrt(mean + eps) and the head's
-// weight and turns adjacent pairs (2i, 2i+1) by the row's angle i. Overlapped
-// sub-tiles are released after their first load as usual and kept in registers;
-// the others are read from tensor memory twice. V heads take the plain path.
+// weight and turns adjacent pairs (2i, 2i+1) by the row's angle i. The angle
+// tables are angle-major ([64, M]): a lane holds one row, so for each angle the
+// warp's 32 rows read one contiguous 128-byte run (row-major tables would cost
+// a cache line per lane and load). Overlapped sub-tiles are released after
+// their first load as usual and kept in registers; the others are read from
+// tensor memory twice. V heads take the plain path.
 #pragma once
 
 #include "sm100.cuh"
@@ -121,7 +124,7 @@ struct GemmParams {
   uint32_t* status;
   // fused QKV epilogue (kQkNorm): q_heads heads of 128 columns each of Q and K
   // (columns [0, 128 q_heads) and [128 q_heads, 256 q_heads)); head weights
-  // [128] bf16 or null (1); rotation tables cos, sin [M, 64] float32 or null
+  // [128] bf16 or null (1); rotation tables cos, sin [64, M] float32 (angle-major) or null
   int q_heads;
   float eps;
   const __nv_bfloat16* norm_q;
@@ -660,7 +663,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           // pass 2: scale, weight, rotate, store. src 0: h0; 1: the parked y; 2: tensor memory
           const float* gamma_s = reinterpret_cast<const float*>(smem + Cfg::kGamma) + (warp - 6) * 128;
           const int m = mrow + quad * 32 + lane;
-          const size_t trow = static_cast<size_t>(m < p.M ? m : 0) * 64;  // rows past M: any valid row
+          const int tcol = m < p.M ? m : 0;  // the row's place in the tables; rows past M: any valid row
           auto emit = [&](int t, int src) {
             const int j0 = sub_col[t];
             float y[32];
@@ -691,21 +694,20 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 y[4 * q4 + 3] = __fmul_rn(__fmul_rn(y[4 * q4 + 3], rs), w.w);
               }
               if (p.rope_cos != nullptr) {
-                // the sub-tile's 16 pairs are angles (j0 mod 128) / 2 .. + 15 of the row
-                const float4* cp = reinterpret_cast<const float4*>(p.rope_cos + trow + ((j0 & 127) >> 1));
-                const float4* sp = reinterpret_cast<const float4*>(p.rope_sin + trow + ((j0 & 127) >> 1));
+                // the sub-tile's 16 pairs are angles a0 .. a0 + 15 of the row, a0 = (j0 mod
+                // 128) / 2; the tables are angle-major, so for each angle the warp's 32
+                // consecutive rows are one contiguous 128-byte run
+                const size_t a0 = static_cast<size_t>((j0 & 127) >> 1) * p.M + tcol;
+                const size_t am = static_cast<size_t>(p.M);
                 auto turn = [](float& a, float& b, float c, float sn) {
                   const float x = a, z = b;
                   a = __fmaf_rn(x, c, -__fmul_rn(z, sn));
                   b = __fmaf_rn(z, c, __fmul_rn(x, sn));
                 };
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  const float4 c = __ldg(cp + q4), sn = __ldg(sp + q4);
-                  turn(y[8 * q4 + 0], y[8 * q4 + 1], c.x, sn.x);
-                  turn(y[8 * q4 + 2], y[8 * q4 + 3], c.y, sn.y);
-                  turn(y[8 * q4 + 4], y[8 * q4 + 5], c.z, sn.z);
-                  turn(y[8 * q4 + 6], y[8 * q4 + 7], c.w, sn.w);
+                for (int i = 0; i < 16; ++i) {
+                  const float c = __ldg(p.rope_cos + a0 + i * am), sn = __ldg(p.rope_sin + a0 + i * am);
+                  turn(y[2 * i], y[2 * i + 1], c, sn);
                 }
               }
             }

@@ -79,9 +79,9 @@ class SvdqQkvNormRope(SvdqW4A4Linear):
     section: to_q, to_k, to_v joined into one SVDQ linear, followed by norm_q / norm_k
     per head and the rotary embedding in one fused call). Weights prepared for the
     joined [3 H 128, K] projection, NVFP4, one-level; norm_q, norm_k bf16 [128] or None.
-    forward(x, rope_cos, rope_sin) takes the rows' angle tables, float32 [M, 64] each
-    (or None: no rotation), and returns Q | K | V [M, 3 H 128], Q and K normalised and
-    rotated."""
+    forward(x, rope_cos, rope_sin) takes the rows' angle tables, float32 [64, M] each,
+    angle-major (or None: no rotation), and returns Q | K | V [M, 3 H 128], Q and K
+    normalised and rotated."""
 
     def __init__(self, weights: dict, bias: torch.Tensor | None, max_tokens: int,
                  norm_q: torch.Tensor | None = None, norm_k: torch.Tensor | None = None,

@@ -297,15 +297,16 @@ svdq_status svdq_mlp_fc1(int M, int N1, int K1, int r1, int r2, const void* a_co
  *   ([128 H, 256 H)) and V ([256 H, 384 H));
  *   each head v of Q and K: z = v * rsqrt(mean(v^2) + eps) * gamma, gamma the
  *   head weight (norm_q for Q, norm_k for K); then each pair (z[2i], z[2i+1]) ->
- *   (z[2i] cos - z[2i+1] sin, z[2i+1] cos + z[2i] sin), cos = rope_cos[m][i] and
- *   sin = rope_sin[m][i];
+ *   (z[2i] cos - z[2i+1] sin, z[2i+1] cos + z[2i] sin), cos = rope_cos[i][m] and
+ *   sin = rope_sin[i][m];
  *   V as svdq_w4a4_linear computes it.
  * All of it in float32 from the accumulator, with one rounding at the output.
  *   N        multiple of 384 (three projections of whole 128-column heads)
  *   norm_q, norm_k  device bf16 [128], 2-byte aligned, or NULL (weight 1)
  *   eps      finite, >= 0 (a head whose values are all zero needs eps > 0)
- *   rope_cos, rope_sin  device float32 [M, 64] row-major (row m: the angles of
- *            token row m), 16-byte aligned; both NULL: no rotation
+ *   rope_cos, rope_sin  device float32 [64, M], angle-major (angle i of token
+ *            row m at i * M + m: the rows an epilogue warp holds read one
+ *            contiguous run per angle), 4-byte aligned; both NULL: no rotation
  * Other arguments, layouts and errors as for svdq_w4a4_linear; INVALID_ARG when
  * N is not a multiple of 384, eps is out of range or only one table is given.
  */

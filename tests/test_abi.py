@@ -71,7 +71,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert g(0, 4, 48, 64, 16, good, good, None, good, good, good, None, good, 48, 0, None) == 1
     assert g(0, 4, 48, 64, 0, good, good, None, good, good, None, None, good, 48, 3, None) == 1
     # the fused QKV epilogue: N a multiple of 384, eps finite and >= 0, both tables or
-    # neither, 16-byte aligned tables, 2-byte aligned head weights
+    # neither, 4-byte aligned tables, 2-byte aligned head weights
     qk = lib.svdq_w4a4_linear_qkv_norm_rope
     eps = ctypes.c_float
 
@@ -82,7 +82,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert qkv(385) == 1 and qkv(256) == 1 and qkv(0) == 1
     assert qkv(384, -1.0) == 1 and qkv(384, float("inf")) == 1 and qkv(384, float("nan")) == 1
     assert qkv(384, cos=good) == 1 and qkv(384, sin=good) == 1
-    assert qkv(384, cos=odd, sin=good) == 2 and qkv(384, cos=good, sin=odd) == 2
+    assert qkv(384, cos=P(0x10002), sin=good) == 2 and qkv(384, cos=good, sin=P(0x10002)) == 2
     assert qkv(384, norm_q=P(0x10001)) == 2
     a = lib.awq_w4a16_linear
     assert a(0, 16, 64, 64, good, good, good, None, good, None) == 1     # M >= 1 (any M above)

@@ -51,10 +51,15 @@ def run_layer(bq, layer, ep, fused: bool, out_f32: bool, weights: bool, rope: bo
                                    K=shape.K, out_dtype=dt)
     gq = C.bf16_tensor(ep["norm_q"]) if weights else None
     gk = C.bf16_tensor(ep["norm_k"]) if weights else None
-    cos = C.f32_tensor(ep["cos"]) if rope else None
-    sin = C.f32_tensor(ep["sin"]) if rope else None
+    cos = angle_major(ep["cos"]) if rope else None
+    sin = angle_major(ep["sin"]) if rope else None
     return bq.svdq_w4a4_linear_qkv_norm_rope(codes, scales, xl1, wc, ws, L2, bias, gq, gk, cos, sin,
                                              shape.M, shape.N, shape.K, eps=1e-6, out_dtype=dt)
+
+
+def angle_major(table):
+    """The oracle's [M, 64] angle table in the call's angle-major [64, M] layout."""
+    return C.f32_tensor(np.ascontiguousarray(table.T))
 
 
 def as_f64(y):
@@ -107,7 +112,7 @@ def test_unit_weights_give_unit_mean_square_heads(bq):
         codes, scales, xl1, C.u8_tensor(C.tiled_codes("nvfp4", layer["w_codes"])),
         C.u8_tensor(C.tiled_scales("nvfp4", layer["w_scales"])),
         C.bf16_tensor(F.bf16_bits(layer["L2"])), C.bf16_tensor(layer["bias_bits"]), None, None,
-        C.f32_tensor(ep["cos"]), C.f32_tensor(ep["sin"]), M, 3 * H * D, K, eps=0.0,
+        angle_major(ep["cos"]), angle_major(ep["sin"]), M, 3 * H * D, K, eps=0.0,
         out_dtype=torch.float32)
     assert bq.svdq_check_device_status() == 0
     heads = as_f64(y)[:, :2 * H * D].reshape(M, 2 * H, D)
@@ -131,7 +136,7 @@ def test_full_size_flux_qkv(bq):
     codes, scales, xl1 = bq.svdq_quantize_act(X, w["L1s"], w["smooth_inv"])
     ep = WL.qkv_epilogue_inputs(M, seed=90, angles="positions")
     gq, gk = C.bf16_tensor(ep["norm_q"]), C.bf16_tensor(ep["norm_k"])
-    cos, sin = C.f32_tensor(ep["cos"]), C.f32_tensor(ep["sin"])
+    cos, sin = angle_major(ep["cos"]), angle_major(ep["sin"])
     y = bq.svdq_w4a4_linear_qkv_norm_rope(codes, scales, xl1, w["w_codes"], w["w_scales"], w["L2"],
                                           bias, gq, gk, cos, sin, M, N, K)
     plain = bq.svdq_w4a4_linear(codes, scales, xl1, w["w_codes"], w["w_scales"], w["L2"], bias,
@@ -178,7 +183,7 @@ def test_layer_class_matches_the_oracle(bq):
          "fmt": "nvfp4", "N": shape.N, "K": K, "r": r}
     mod = SvdqQkvNormRope(w, C.bf16_tensor(layer["bias_bits"]), max_tokens=512,
                           norm_q=C.bf16_tensor(ep["norm_q"]), norm_k=C.bf16_tensor(ep["norm_k"]))
-    y = mod(C.bf16_tensor(layer["x_bits"]), C.f32_tensor(ep["cos"]), C.f32_tensor(ep["sin"]))
+    y = mod(C.bf16_tensor(layer["x_bits"]), angle_major(ep["cos"]), angle_major(ep["sin"]))
     assert bq.svdq_check_device_status() == 0
     fwd = S.svdq_forward("nvfp4", layer["x_bits"], layer["smooth_inv"], layer["L1"], layer["L2"],
                          layer["w_codes"], layer["w_scales"], layer["bias_bits"])

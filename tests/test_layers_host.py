@@ -61,7 +61,7 @@ def test_qkv_layer_routes_its_workspaces_and_epilogue_inputs(monkeypatch):
     layer = L.SvdqQkvNormRope(weights(N, K, r), None, max_tokens=300, norm_q=gq, norm_k=gk, eps=1e-5)
     assert layer.heads == 2
     x = torch.zeros(260, K, dtype=BF)
-    cos, sin = torch.zeros(260, 64), torch.zeros(260, 64)
+    cos, sin = torch.zeros(64, 260), torch.zeros(64, 260)
     assert layer(x, cos, sin) == "Y"
     (q, M, codes, scales, xl1), g = rec.calls
     assert q == "quantize" and M == 260 and codes is layer.codes and scales is layer.scales
