@@ -667,6 +667,18 @@ def main() -> None:
     k2_ms = sum(b[0].elapsed_time(b[1]) for b in ev_k) / args.steps
     k3_ms = sum(b[1].elapsed_time(e) for b, e in zip(ev_k, ev_ke)) / args.steps
     status = bq.svdq_check_device_status()
+    # The event floor: a one-element torch kernel timed the same way (flush, event,
+    # kernel, event). Every event-to-event figure above carries it; for the short
+    # kernels it is a large part of their time.
+    tiny = torch.zeros(1, device=dev)
+    ev_f = [(mk(), mk()) for _ in range(args.steps + 3)]
+    for i in range(args.steps + 3):
+        flush()
+        ev_f[i][0].record(stream)
+        tiny.add_(1.0)
+        ev_f[i][1].record(stream)
+    torch.cuda.synchronize()
+    floor_ms = sorted(a.elapsed_time(b) for a, b in ev_f[3:])[args.steps // 2]
 
     # ------------------------------ two-level NVFP4 on the same layer (per-tensor scales)
     # The same X and weights, quantized with a per-tensor float32 scale above the
@@ -825,7 +837,9 @@ def main() -> None:
                 "algorithmic_bytes": quantize_bytes(M, K, r),
                 "traffic": sum_traffic(("quantize_act_kernel", "xl1_reduce_kernel")),
                 "kernels": "quantize_act_kernel + xl1_reduce_kernel (K-split partial sums)",
-                "us": k1_ms * 1e3},
+                "us": k1_ms * 1e3,
+                "frac_net_of_event_floor": quantize_bytes(M, K, r) / ((k1_ms - floor_ms) * 1e-3) / 1e9
+                / peaks["hbm_gbs"]},
             "awq_w4a16_linear": {
                 "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "achieved": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / (k3_ms * 1e-3) / 1e9,
@@ -833,9 +847,14 @@ def main() -> None:
                 "algorithmic_bytes": awq_bytes(AWQ.M, AWQ.K, AWQ.N),
                 "traffic": sum_traffic((AWQ_KERNEL,)),
                 "kernels": AWQ_KERNEL,
-                "us": k3_ms * 1e3},
+                "us": k3_ms * 1e3,
+                "frac_net_of_event_floor": awq_bytes(AWQ.M, AWQ.K, AWQ.N) / ((k3_ms - floor_ms) * 1e-3) / 1e9
+                / peaks["hbm_gbs"]},
+            "event_floor_us": floor_ms * 1e3,
             "peak_note": f"{peaks['source']} HBM copy bandwidth; achieved = algorithmic bytes / "
-                         f"event-to-event time in the kernel-timing pass"},
+                         f"event-to-event time in the kernel-timing pass; frac_net_of_event_floor "
+                         f"takes event_floor_us (a one-element torch kernel timed the same way, "
+                         f"flush, event, kernel, event) off that time"},
         "cpu_baseline": cpu,
         "e2e": {"value": job_tflops(step_flops(), world, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2 + Xa.numel() * 2,
