@@ -103,3 +103,21 @@ def test_xl1_splits_is_a_pure_function_of_the_shape(lib):
     assert lib.svdq_xl1_splits(4608, 3072, 0) == 1       # no low-rank branch
     assert lib.svdq_xl1_splits(4608, 3000, 32) == 0      # K not a multiple of 64
     assert lib.svdq_xl1_splits(4608, 3072, 24) == 0      # rank not a multiple of 16
+
+
+def test_binding_takes_the_rotary_tables_angle_major(lib):
+    """The fused QKV call's cos/sin tables are [64, M] (angle i of row m at
+    i * M + m); the binding refuses row-major [M, 64] tables before any device
+    work, whatever M is."""
+    import torch
+    import bit_quantized_diffusion_b200 as bq
+    M, N, K = 100, 384, 128
+    codes = torch.zeros(M * K // 2, dtype=torch.uint8)
+    scales = torch.zeros(M * K // 16, dtype=torch.uint8)
+    wc = torch.zeros(N * K // 2, dtype=torch.uint8)
+    ws = torch.zeros(N * K // 16, dtype=torch.uint8)
+    for shape in ((M, 64), (64, M + 1), (64 * M,)):
+        t = torch.zeros(shape, dtype=torch.float32)
+        with pytest.raises(ValueError, match="angle-major"):
+            bq.svdq_w4a4_linear_qkv_norm_rope(codes, scales, None, wc, ws, None, None, None, None, t, t,
+                                              M, N, K)
