@@ -683,15 +683,21 @@ __global__ void __launch_bounds__(kGmThreads, 1)
               finish(acc, t, y);
             }
             if (n0 / 128 + (j0 >> 7) < 2 * p.q_heads) {
+              // paired float32 instructions; each lane rounds as the scalar form would
               const float rs = j0 < 128 ? rs0 : rs1;
+              const float2 rs2 = make_float2(rs, rs);
               const float4* gv = reinterpret_cast<const float4*>(gamma_s + t * 32);
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4) {
                 const float4 w = gv[q4];
-                y[4 * q4 + 0] = __fmul_rn(__fmul_rn(y[4 * q4 + 0], rs), w.x);
-                y[4 * q4 + 1] = __fmul_rn(__fmul_rn(y[4 * q4 + 1], rs), w.y);
-                y[4 * q4 + 2] = __fmul_rn(__fmul_rn(y[4 * q4 + 2], rs), w.z);
-                y[4 * q4 + 3] = __fmul_rn(__fmul_rn(y[4 * q4 + 3], rs), w.w);
+                const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(y[4 * q4 + 0], y[4 * q4 + 1]), rs2),
+                                             make_float2(w.x, w.y));
+                const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(y[4 * q4 + 2], y[4 * q4 + 3]), rs2),
+                                             make_float2(w.z, w.w));
+                y[4 * q4 + 0] = lo.x;
+                y[4 * q4 + 1] = lo.y;
+                y[4 * q4 + 2] = hi.x;
+                y[4 * q4 + 3] = hi.y;
               }
               if (p.rope_cos != nullptr) {
                 // the sub-tile's 16 pairs are angles a0 .. a0 + 15 of the row, a0 = (j0 mod
@@ -699,15 +705,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 // consecutive rows are one contiguous 128-byte run
                 const size_t a0 = static_cast<size_t>((j0 & 127) >> 1) * p.M + tcol;
                 const size_t am = static_cast<size_t>(p.M);
-                auto turn = [](float& a, float& b, float c, float sn) {
-                  const float x = a, z = b;
-                  a = __fmaf_rn(x, c, -__fmul_rn(z, sn));
-                  b = __fmaf_rn(z, c, __fmul_rn(x, sn));
-                };
+                // (x, z) -> (x c - RN(z s), z c + RN(x s)): the products (-z s, x s) as one
+                // paired multiply, then one paired fused multiply-add
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                   const float c = __ldg(p.rope_cos + a0 + i * am), sn = __ldg(p.rope_sin + a0 + i * am);
-                  turn(y[2 * i], y[2 * i + 1], c, sn);
+                  const float2 zx = __fmul2_rn(make_float2(y[2 * i + 1], y[2 * i]), make_float2(-sn, sn));
+                  const float2 r = __ffma2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(c, c), zx);
+                  y[2 * i] = r.x;
+                  y[2 * i + 1] = r.y;
                 }
               }
             }
