@@ -20,10 +20,11 @@
 // so a pair of codes dequantizes with one byte select, one mask, one FP16
 // subtract and one FP16 multiply.
 //
-// Persistent kernel. In pair mode (kPair) a cluster of two CTAs on two SMs
-// computes 256 x 256 output tiles with cta_group::2 MMAs: each CTA dequantizes
-// its own 128 rows of A and 128 of the tile's 256 B rows, and each CTA's tensor
-// memory accumulates its 128 rows. Without kPair one CTA computes 128 x 256.
+// Persistent kernel. A cluster of two CTAs on two SMs computes 256 x 256 output
+// tiles with cta_group::2 MMAs: each CTA dequantizes its own 128 rows of A and
+// 128 of the tile's 256 B rows, and each CTA's tensor memory accumulates its 128
+// rows. The kernel is launched in pairs only (kPair): a lone CTA's converters
+// would fill only half of the 256 B rows its N = 256 MMAs read.
 // Two disjoint 256-column accumulators (no scale factors live in tensor
 // memory) let the next tile's MMAs run while the epilogue drains the last one.
 //
@@ -120,6 +121,7 @@ __global__ void __maxnreg__(80)
                           const __grid_constant__ CUtensorMap tm_l2,
                           const __grid_constant__ CUtensorMap tm_y, const I4Params p) {
   constexpr int kCtas = kPair ? 2 : 1;
+  static_assert(kPair, "CTA pairs only: a lone CTA's converters fill 128 of the tile's 256 B rows");
   constexpr int NP = kI4PkStages, NO = kI4OpStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

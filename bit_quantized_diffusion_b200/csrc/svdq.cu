@@ -130,9 +130,7 @@ svdq_status device_setup(DeviceInfo** out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(GmCfg<true, true>::kSmemBytes)) != cudaSuccess)
       return SVDQ_ERR_CUDA;
-    if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
-        cudaFuncSetAttribute(w4a4_int4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a4_int4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kI4SmemBytes)) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_mlp_fc1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMlSmemBytes)) != cudaSuccess)
@@ -145,7 +143,6 @@ svdq_status device_setup(DeviceInfo** out) {
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<false, true>),
                           reinterpret_cast<const void*>(w4a4_nvfp4_gemm_kernel<true, true>),
-                          reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<false>),
                           reinterpret_cast<const void*>(w4a4_int4_gemm_kernel<true>),
                           reinterpret_cast<const void*>(awq_gemm_kernel),
                           reinterpret_cast<const void*>(w4a4_mlp_fc1_kernel),
@@ -260,14 +257,15 @@ unsigned grid_for(size_t n, unsigned threads) {
 
 // INT4 W4A4 GEMM (w4a4_int4_gemm_kernel): packed codes [rows, K/2] as one-group
 // boxes [128 rows x 32 B], group-major FP16 scales [K/64][rows padded to 128]
-// as one-group boxes [128], Y as 32 x 32 TMA-store boxes. CTA pairs whenever M
-// exceeds one 128-row block, as for NVFP4.
+// as one-group boxes [128], Y as 32 x 32 TMA-store boxes. Always CTA pairs, at
+// any M: each CTA's converters fill 128 of a tile's 256 weight rows, so one CTA
+// alone would leave half of the tile's B operand unfilled. Rows of a pair's tile
+// past M read as zeros (TMA fill) and are clipped by the TMA store.
 svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, const void* a_codes,
                              const void* a_scales, const float* xl1, const void* w_codes,
                              const void* w_scales, const void* L2, const void* bias, void* Y,
                              int ldy, svdq_out out, cudaStream_t stream) {
-  const bool pair = (d->gemm_pair_mode < 0 ? true : d->gemm_pair_mode != 0) && M > kI4BM;
-  const int ctas = pair ? 2 : 1;
+  const int ctas = 2;
   CUtensorMap tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y;
   const uint64_t G = static_cast<uint64_t>(K / 64);
   if (!make_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 32, kI4BM,
@@ -304,13 +302,9 @@ svdq_status launch_int4_gemm(const DeviceInfo* d, int M, int N, int K, int r, co
   p.status = d->status;
   p.tiles_m = (M + kI4BM * ctas - 1) / (kI4BM * ctas);
   p.tiles = p.tiles_m * ((N + kI4BN - 1) / kI4BN);
-  const int max_units = pair ? d->int4_pairs : d->num_sms;
-  const int units = p.tiles < max_units ? p.tiles : max_units;
-  const cudaError_t e =
-      pair ? launch_kernel(d, w4a4_int4_gemm_kernel<true>, dim3(units * 2), dim3(kI4Threads),
-                           kI4SmemBytes, stream, 2, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p)
-           : launch_kernel(d, w4a4_int4_gemm_kernel<false>, dim3(units), dim3(kI4Threads),
-                           kI4SmemBytes, stream, 1, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p);
+  const int units = p.tiles < d->int4_pairs ? p.tiles : d->int4_pairs;
+  const cudaError_t e = launch_kernel(d, w4a4_int4_gemm_kernel<true>, dim3(units * 2), dim3(kI4Threads),
+                                      kI4SmemBytes, stream, 2, tm_a, tm_b, tm_sa, tm_sw, tm_l2, tm_y, p);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SVDQ_ERR_CUDA;

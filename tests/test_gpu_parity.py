@@ -50,6 +50,11 @@ SMALL_INT4 = [
     WL.custom_svdq("int4_r0", 130, 256, 160, 0, fmt="int4", seed=26),
     WL.custom_svdq("int4_r256", 200, 512, 256, 256, fmt="int4", seed=27, spike_rank=8, spike_sv=5.0),
     WL.custom_svdq("int4_many_tiles_r128", 2176, 256, 2560, 128, fmt="int4", seed=28),
+    # at most 128 rows with more than 128 columns per tile: the CTA pair's second CTA holds
+    # only rows past M, and the tile's second 128 weight rows must still be converted
+    WL.custom_svdq("int4_few_rows_wide", 100, 640, 400, 32, fmt="int4", seed=29),
+    WL.custom_svdq("int4_one_row_wide", 1, 256, 272, 16, fmt="int4", seed=30),
+    WL.custom_svdq("int4_128_rows", 128, 512, 528, 48, fmt="int4", seed=31),
 ]
 
 
