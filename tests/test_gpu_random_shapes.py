@@ -2,8 +2,8 @@
 the quantizer's codes and scales bit-exact and the W4A4 linear within the
 stated tolerance of the oracle (both formats, M from 1 row to several tiles,
 any N % 16, K % 64 and r % 16 within the supported ranges), the fused QKV
-projection, and the AWQ linear on either of its kernels. The shapes are drawn
-once from a fixed seed, so a failure names a reproducible case."""
+projection, the AWQ linear on either of its kernels, and the fused MLP. The
+shapes are drawn once from a fixed seed, so a failure names a reproducible case."""
 
 import numpy as np
 import pytest
@@ -11,6 +11,7 @@ import pytest
 import workloads as WL
 from tests import svdq_cases as C
 from tests import test_gpu_awq_gemm as TA
+from tests import test_gpu_mlp as TM
 from tests import test_gpu_parity as TP
 from tests import test_gpu_qkv_epilogue as TQ
 
@@ -28,6 +29,13 @@ QKV = [(int(_rng.integers(1, 900)), int(_rng.integers(1, 5)), int(_rng.integers(
         bool(_rng.integers(0, 2))) for _ in range(6)]
 AWQ = [(int(_rng.integers(1, 300)), int(_rng.integers(1, 40)) * 16, int(_rng.integers(1, 17)) * 64,
         bool(_rng.integers(0, 2))) for _ in range(6)]
+# fused MLP: N1 % 128, r2 in {0, 32, 64, 96, 128} and at most fc2's width N2
+MLP = []
+while len(MLP) < 5:
+    _m = (int(_rng.integers(1, 1500)), int(_rng.integers(1, 17)) * 64, int(_rng.integers(1, 13)) * 128,
+          int(_rng.integers(1, 33)) * 16, int(_rng.choice([0, 16, 32, 64])), int(_rng.choice([0, 32, 64, 96, 128])))
+    if _m[5] <= _m[3]:
+        MLP.append(_m)
 
 
 @pytest.fixture(scope="module")
@@ -55,3 +63,10 @@ def test_random_awq(bq, M, N, K, bias):
     x_bits, q, s, z, b_bits, ref = TA._case(M, N, K, 9000 + M + N, bias)
     y = TA._run(bq, x_bits, q, s, z, b_bits, None)
     C.assert_gemm_close(y, ref, bf16_out=True, what="AWQ Y")
+
+
+@pytest.mark.parametrize("M,K1,N1,N2,r1,r2", MLP, ids=lambda v: str(v))
+def test_random_fused_mlp(bq, M, K1, N1, N2, r1, r2):
+    d1, p1, d2, p2 = TM._layers(M, K1, N1, N2, r1, r2, seed=7000 + M)
+    out = TM._run(bq, d1, p1, d2, p2, M, K1, N1, N2, r1, r2)
+    TM._check(bq, out, d1, p1, d2, p2, M, r2)
